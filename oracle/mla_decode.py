@@ -1,0 +1,227 @@
+"""fp64 CPU oracle for MLA decode in absorbed latent space.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, links or
+executes this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may use it.  It
+shares no code with the CUDA path.
+
+What it computes (page "MLA Cost Analysis & Regime Guide", section
+"Absorption Trick"): with the key and value projections absorbed, every head
+scores against the shared latent cache directly,
+
+    score  = Qz . Z^T          (Qz = the absorbed 576-d query row, Z = cache rows)
+    value  = softmax(score) . Z[:, :512]
+
+which is exactly ordinary softmax attention whose keys are the 576-d cache
+rows and whose values are their first 512 entries.  So the oracle is that
+plain definition, written out per (request, query token), in float64:
+
+  1. L = t_r - s + i + 1 for query token i of a causal speculative step
+     (query i sees keys j <= t_r - s + i); L = t_r otherwise.
+  2. C_j = cache row j (j < L) gathered through the block table:
+     pool[block_table[r][j // 64], j % 64, :].  For the FP8 cache,
+     C_j[:512] = e4m3(byte) * scale_j and C_j[512:] = the bf16 RoPE part.
+  3. x_j = softmax_scale * sum_d Q[r, i, h, d] * C_j[d]
+  4. lse = m + ln sum_j exp(x_j - m), m = max_j x_j
+  5. O[r, i, h, c] = sum_j exp(x_j - lse) * C_j[c], c < 512.
+
+L <= 0 gives O = 0 and lse = -inf.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+PAGE = 64
+D_QK = 576
+D_V = 512
+
+
+# ----------------------------------------------------------------------------
+# element decoding
+# ----------------------------------------------------------------------------
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    """bf16 -> float64, exact (bf16 is the top half of an IEEE binary32)."""
+    bits = t.contiguous().view(torch.int16).numpy().astype(np.uint16).astype(np.uint32) << 16
+    return bits.view(np.float32).astype(np.float64)
+
+
+def e4m3_table() -> np.ndarray:
+    """Value of every e4m3 ("fn" variant: no infinities) byte, from the
+    format's definition: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent 0 is subnormal (2^-6 * m/8); S.1111.111 is NaN."""
+    tab = np.empty(256, dtype=np.float64)
+    for byte in range(256):
+        sign = -1.0 if byte & 0x80 else 1.0
+        e = (byte >> 3) & 0xF
+        m = byte & 0x7
+        if e == 0xF and m == 0x7:
+            tab[byte] = np.nan
+        elif e == 0:
+            tab[byte] = sign * math.ldexp(m / 8.0, -6)
+        else:
+            tab[byte] = sign * math.ldexp(1.0 + m / 8.0, e - 7)
+    return tab
+
+
+_E4M3 = e4m3_table()
+
+
+def page_rows_f64(pool, page: int, kv_scale=None) -> np.ndarray:
+    """One 64-token page as float64 rows [64, 576].
+
+    ``pool`` is bf16 [P, 64, 576], or uint8 [P, 40960] for the FP8 cache whose
+    page holds 64x512 e4m3 bytes then 64x64 bf16 RoPE values; the fp32
+    per-token scales come in ``kv_scale`` [P, 64]."""
+    if pool.dtype == torch.bfloat16:
+        return bf16_to_f64(pool[page])
+    raw = pool[page].numpy()
+    lat = _E4M3[raw[:PAGE * D_V].reshape(PAGE, D_V)]
+    sc = kv_scale[page].numpy().astype(np.float64)
+    rope = bf16_to_f64(torch.from_numpy(raw[PAGE * D_V:].copy()).view(torch.bfloat16)).reshape(PAGE, D_QK - D_V)
+    out = np.empty((PAGE, D_QK), dtype=np.float64)
+    out[:, :D_V] = lat * sc[:, None]
+    out[:, D_V:] = rope
+    return out
+
+
+def gather_rows(pool, block_table, r: int, n: int, kv_scale=None, start: int = 0) -> np.ndarray:
+    """Cache rows start..start+n-1 of request r as float64 [n, 576]."""
+    out = np.empty((max(n, 0), D_QK), dtype=np.float64)
+    j = start
+    while j < start + n:
+        pg = int(block_table[r][j // PAGE])
+        rows = page_rows_f64(pool, pg, kv_scale)
+        lo = j % PAGE
+        hi = min(PAGE, lo + (start + n - j))
+        out[j - start:j - start + hi - lo] = rows[lo:hi]
+        j += hi - lo
+    return out
+
+
+def visible_len(t: int, s_q: int, i: int, causal: bool) -> int:
+    """Keys seen by query token i (step 1 of the definition)."""
+    return t - s_q + i + 1 if causal else t
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+
+def attend(qrows: np.ndarray, C: np.ndarray, scale: float):
+    """Plain softmax attention of query rows [h, 576] over cache rows
+    [L, 576] (steps 3-5).  Returns (O [h, 512], lse [h]) in float64."""
+    h = qrows.shape[0]
+    if C.shape[0] == 0:
+        return np.zeros((h, D_V)), np.full(h, -np.inf)
+    x = scale * (qrows @ C.T)                       # [h, L]
+    m = x.max(axis=1, keepdims=True)
+    lse = m[:, 0] + np.log(np.exp(x - m).sum(axis=1))
+    w = np.exp(x - lse[:, None])
+    return w @ C[:, :D_V], lse
+
+
+def decode(wl, rows=None):
+    """Oracle over a whole workload (or over selected (r, i) query tokens).
+
+    ``wl`` carries q bf16 [b, s, h, 576], pool, kv_scale, block_table,
+    seqlens, softmax_scale, s_q and causal.  ``rows`` optionally lists
+    (r, i) pairs; the result then has shape [len(rows), h, 512] / [len(rows), h].
+    Returns (O float64 [b, s, h, 512], lse float64 [b, s, h])."""
+    b, s, h, _ = wl.q.shape
+    sel = [(r, i) for r in range(b) for i in range(s)] if rows is None else list(rows)
+    O = np.zeros((len(sel), h, D_V))
+    L = np.zeros((len(sel), h))
+    cache = {}
+    for n, (r, i) in enumerate(sel):
+        t = int(wl.seqlens[r])
+        Lv = visible_len(t, s, i, wl.causal)
+        if r not in cache:
+            cache = {r: gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale)}
+        C = cache[r][:max(Lv, 0)]
+        q = bf16_to_f64(wl.q[r, i])
+        O[n], L[n] = attend(q, C, wl.softmax_scale)
+    if rows is None:
+        return O.reshape(b, s, h, D_V), L.reshape(b, s, h)
+    return O, L
+
+
+def decode_chunk(wl, r: int, i: int, start: int, stop: int):
+    """Attention of query token (r, i) over its visible keys in [start, stop)
+    only: the partial result one split of a split-KV schedule produces."""
+    t = int(wl.seqlens[r])
+    Lv = visible_len(t, wl.s_q, i, wl.causal)
+    stop = min(stop, Lv)
+    C = gather_rows(wl.pool, wl.block_table, r, max(stop - start, 0), wl.kv_scale, start=start)
+    return attend(bf16_to_f64(wl.q[r, i]), C, wl.softmax_scale)
+
+
+def combine(parts):
+    """Merge partial (O_i, lse_i) results over disjoint key ranges:
+    L = ln sum_i e^{lse_i};  O = sum_i e^{lse_i - L} O_i."""
+    lses = np.stack([p[1] for p in parts])          # [n, h]
+    m = lses.max(axis=0)
+    finite = np.isfinite(m)
+    msafe = np.where(finite, m, 0.0)
+    w = np.exp(lses - msafe)                        # e^{-inf} = 0
+    tot = w.sum(axis=0)
+    L = np.where(finite, msafe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    O = np.zeros_like(parts[0][0])
+    for (Oi, li) in parts:
+        wi = np.where(finite, np.exp(li - np.where(finite, L, 0.0)), 0.0)
+        O += wi[:, None] * Oi
+    return O, L
+
+
+def brute(wl):
+    """Triple loop in pure Python (tiny inputs only): every score, max,
+    exponential and weighted sum written out one element at a time, the
+    cache read token by token through the block table."""
+    b, s, h, _ = wl.q.shape
+    O = np.zeros((b, s, h, D_V))
+    LSE = np.zeros((b, s, h))
+    for r in range(b):
+        t = int(wl.seqlens[r])
+        for i in range(s):
+            Lv = visible_len(t, s, i, wl.causal)
+            rows = []
+            for j in range(max(Lv, 0)):
+                page = int(wl.block_table[r][j // PAGE])
+                rows.append(page_rows_f64(wl.pool, page, wl.kv_scale)[j % PAGE].tolist())
+            for hh in range(h):
+                q = bf16_to_f64(wl.q[r, i, hh]).tolist()
+                if not rows:
+                    LSE[r, i, hh] = -math.inf
+                    continue
+                xs = []
+                for row in rows:
+                    acc = 0.0
+                    for d in range(D_QK):
+                        acc += q[d] * row[d]
+                    xs.append(wl.softmax_scale * acc)
+                mx = max(xs)
+                z = sum(math.exp(x - mx) for x in xs)
+                lse = mx + math.log(z)
+                LSE[r, i, hh] = lse
+                for c in range(D_V):
+                    acc = 0.0
+                    for x, row in zip(xs, rows):
+                        acc += math.exp(x - lse) * row[c]
+                    O[r, i, hh, c] = acc
+    return O, LSE
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 (ties to even), returned as
+    float64: the comparison target for bf16 kernel outputs."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                               # x = m 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)                          # below 2^-126: fixed subnormal spacing
+    ulp = np.ldexp(1.0, e - 8)                       # 8 significant bits
+    with np.errstate(invalid="ignore", over="ignore"):
+        r = np.round(x / ulp) * ulp                  # np.round: ties to even
+        r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, x), r)
+    return np.where(np.isfinite(x), r, x)

@@ -1,0 +1,316 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself
+(values printed on the pages, closed forms, a library routine, brute force).
+
+Citations name the "MLA Cost Analysis & Regime Guide" page (sections "Cost
+Models", "Absorption Trick", "Tensor Shapes", "Historical Baselines") and the
+FlashMLA-2 newsletter page (section "Architectural Analysis": split-KV
+balancing across SMs).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import mla_decode as om
+import mla_workloads as mw
+from mla_workloads import cost
+from conftest import load_golden
+
+SCALE = 1.0 / math.sqrt(192.0)
+
+
+# --------------------------------------------------------------------------
+# cost model vs the numbers the page prints ("Cost Models")
+# --------------------------------------------------------------------------
+
+def test_cost_model_matches_printed_values():
+    g = load_golden("cost_model.txt")
+    b, h, t, k, p, d = 64, 128, 4096, 512, 64, 128
+    ai = cost.mla_flops(b, h, 1, t) / cost.mla_bytes(b, h, 1, t)
+    assert abs(ai - g["flashmla_ai_s1"][0]) <= g["flashmla_ai_s1"][1]
+    fa1 = cost.fa_flops(b, h, 1, t) / cost.fa_bytes(b, h, 1, t)
+    assert abs(fa1 - g["fa_ai_s1"][0]) <= g["fa_ai_s1"][1]
+    fa1024 = cost.fa_flops(b, h, 1024, t) / cost.fa_bytes(b, h, 1024, t)
+    assert abs(fa1024 - g["fa_ai_s1024"][0]) <= g["fa_ai_s1024"][1]
+    # per-token FLOP factors 2k+p and 2d+p, and their ratio
+    assert cost.mla_flops(1, 1, 1, 1) / 2 == g["flashmla_flop_factor"][0]
+    assert cost.fa_flops(1, 1, 1, 1) / 2 == g["fa_flop_factor"][0]
+    ratio = cost.mla_flops(b, h, 1, t) / cost.fa_flops(b, h, 1, t)
+    assert abs(ratio - g["flops_per_token_ratio"][0]) <= g["flops_per_token_ratio"][1]
+    # the recomputed value the roofline uses (no rounding): 228.30
+    assert abs(ai - 228.30) < 0.01
+
+
+def test_cost_model_batch_independence_and_jagged_sum():
+    # AI at s=1 does not depend on b; a jagged batch sums its lengths
+    a1 = cost.mla_flops(1, 128, 1, 4096) / cost.mla_bytes(1, 128, 1, 4096)
+    a2 = cost.mla_flops(64, 128, 1, 4096) / cost.mla_bytes(64, 128, 1, 4096)
+    assert abs(a1 - a2) < 1e-9
+    assert cost.mla_flops(3, 128, 1, None, sum_t=100 + 200 + 300) == cost.mla_flops(3, 128, 1, 200)
+
+
+def test_mlavar6_flops_interpolate_between_the_two_models():
+    # the split-cache design reduces to the latent model at n=0 and to the
+    # decompressed model at o=0 ("MLAvar6+ Design")
+    b, h, s, t = 32, 128, 16, 4096
+    assert cost.mlavar6_flops(b, h, s, t, 0) == cost.mla_flops(b, h, s, t)
+    assert cost.mlavar6_flops(b, h, s, 0, t) == cost.fa_flops(b, h, s, t)
+
+
+def test_latency_table_ratios():
+    g = load_golden("rtx5090_latency_table.txt")
+    sp = g["fa_s1_us"][0] / g["flashmla_s1_us"][0]
+    assert abs(sp - g["decode_speedup_vs_fa"][0]) <= g["decode_speedup_vs_fa"][1]
+    gain = 100.0 * (g["flashmla_s16_us"][0] - g["mlavar6_v3_s16_us"][0]) / g["flashmla_s16_us"][0]
+    assert abs(gain - g["mlavar6_gain_s16_pct"][0]) <= g["mlavar6_gain_s16_pct"][1]
+
+
+# --------------------------------------------------------------------------
+# element decoding vs library conversions
+# --------------------------------------------------------------------------
+
+def test_e4m3_table_matches_torch():
+    tab = om.e4m3_table()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(tab))
+    assert np.array_equal(tab[~nan], ref[~nan])
+    assert tab[0x7E] == 448.0 and tab[0x01] == 2.0 ** -9
+
+
+def test_bf16_decode_matches_torch():
+    g = torch.Generator().manual_seed(1)
+    x = (torch.randn(4096, generator=g) * 100).to(torch.bfloat16)
+    x[:4] = torch.tensor([0.0, -0.0, 1e-40, -3e38]).to(torch.bfloat16)
+    assert np.array_equal(om.bf16_to_f64(x), x.to(torch.float64).numpy())
+
+
+def test_round_bf16_matches_torch_rne():
+    g = torch.Generator().manual_seed(2)
+    f = torch.randn(100000, generator=g, dtype=torch.float32) * 3
+    f[:3] = torch.tensor([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8)])  # exact ties
+    ref = f.to(torch.bfloat16).to(torch.float64).numpy()
+    got = om.round_bf16(f.to(torch.float64).numpy())
+    assert np.array_equal(ref, got)
+
+
+# --------------------------------------------------------------------------
+# attention: brute force, closed forms, library routine
+# --------------------------------------------------------------------------
+
+def _tiny(seqlens, h=4, s_q=1, causal=False, cache_dtype="bf16", seed=3, contiguous=False):
+    return mw.make(len(seqlens), s_q, h, list(seqlens), causal=causal, cache_dtype=cache_dtype,
+                   seed=seed, contiguous=contiguous)
+
+
+@pytest.mark.parametrize("lens", [[1], [63], [64], [65], [1, 130, 64]])
+def test_vectorised_matches_brute_force(lens):
+    wl = _tiny(lens, h=3)
+    O, L = oracle.decode(wl)
+    Ob, Lb = oracle.brute(wl)
+    assert np.max(np.abs(O - Ob)) < 1e-12
+    assert np.max(np.abs(L - Lb)) < 1e-12
+
+
+def test_brute_force_causal_and_fp8():
+    wl = _tiny([70, 5], h=2, s_q=3, causal=True)
+    O, L = oracle.decode(wl)
+    Ob, Lb = oracle.brute(wl)
+    assert np.max(np.abs(O - Ob)) < 1e-12 and np.max(np.abs(L - Lb)) < 1e-12
+    wl8 = _tiny([67], h=2, cache_dtype="fp8")
+    O, L = oracle.decode(wl8)
+    Ob, Lb = oracle.brute(wl8)
+    assert np.max(np.abs(O - Ob)) < 1e-12 and np.max(np.abs(L - Lb)) < 1e-12
+
+
+def test_brute_force_config1_shape():
+    # the tiny workload's exact shape (b=2, h=16, t=256, contiguous), two heads
+    # checked by brute force to keep the pure-Python loop short
+    wl = mw.make_config(1)
+    O, L = oracle.decode(wl)
+    sub = mw.make(2, 1, 16, 256, contiguous=True, seed=0)
+    sub.q = sub.q[:, :, :2].contiguous()
+    Ob, Lb = oracle.brute(sub)
+    assert np.max(np.abs(O[:, :, :2] - Ob)) < 1e-12 and np.max(np.abs(L[:, :, :2] - Lb)) < 1e-12
+
+
+def _absorption_case(seed=0, t=96, h=4):
+    """Random DeepSeek-style factors: per head W_k, W_v (k x d), q_nope (d),
+    q_pe (p); a latent cache Z (t x k) and RoPE keys KPE (t x p)."""
+    g = torch.Generator().manual_seed(seed)
+    k, d, p = 512, 128, 64
+    Wk = torch.randn(h, k, d, generator=g, dtype=torch.float64) / math.sqrt(k)
+    Wv = torch.randn(h, k, d, generator=g, dtype=torch.float64) / math.sqrt(k)
+    qn = torch.randn(h, d, generator=g, dtype=torch.float64)
+    qp = torch.randn(h, p, generator=g, dtype=torch.float64)
+    Z = torch.randn(t, k, generator=g, dtype=torch.float64)
+    KPE = torch.randn(t, p, generator=g, dtype=torch.float64)
+    return Wk, Wv, qn, qp, Z, KPE
+
+
+def _mha_reference(Wk, Wv, qn, qp, Z, KPE):
+    """Ordinary multi-head attention with decompressed per-head keys
+    K_h = [Z Wk_h | KPE] and values V_h = Z Wv_h, through the library's
+    scaled_dot_product_attention in float64, scale 1/sqrt(d + p)."""
+    h = Wk.shape[0]
+    K = torch.stack([torch.cat([Z @ Wk[i], KPE], dim=1) for i in range(h)])      # h, t, 192
+    V = torch.stack([Z @ Wv[i] for i in range(h)])                               # h, t, 128
+    Q = torch.cat([qn, qp], dim=1)[:, None, :]                                   # h, 1, 192
+    return torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=SCALE)[:, 0]
+
+
+def _latent_path(attend, Wk, Wv, qn, qp, Z, KPE):
+    """Absorbed path: Qz_h = [Wk_h qn_h | qp_h], cache rows [Z | KPE], the
+    oracle's attention, then decompression O_lat,h Wv_h."""
+    h = Wk.shape[0]
+    Qz = torch.stack([torch.cat([Wk[i] @ qn[i], qp[i]]) for i in range(h)]).numpy()
+    C = torch.cat([Z, KPE], dim=1).numpy()
+    Olat, _ = attend(Qz, C, SCALE)
+    return np.stack([Olat[i] @ Wv[i].numpy() for i in range(h)])
+
+
+def test_absorption_identity():
+    case = _absorption_case()
+    ref = _mha_reference(*case).numpy()
+    got = _latent_path(oracle.attend, *case)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_uniform_scores_give_mean_of_values():
+    # Q = 0: every score is 0, so the weights are 1/L, O is the mean of the
+    # value rows and lse = ln L
+    wl = _tiny([1, 77, 200], h=2)
+    wl.q.zero_()
+    O, L = oracle.decode(wl)
+    for r, t in enumerate(wl.seqlens):
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        assert np.max(np.abs(O[r, 0] - C[:, :512].mean(axis=0))) < 1e-12
+        assert np.max(np.abs(L[r, 0] - math.log(t))) < 1e-12
+
+
+def test_rows_sum_to_one():
+    # a latent column that is 1 in every cache row must come out as exactly 1
+    wl = _tiny([150, 3], h=4)
+    wl.pool[:, :, 17] = 1.0
+    O, _ = oracle.decode(wl)
+    assert np.max(np.abs(O[..., 17] - 1.0)) < 1e-12
+
+
+def test_single_key_returns_its_value():
+    wl = _tiny([1], h=4)
+    O, L = oracle.decode(wl)
+    C = om.gather_rows(wl.pool, wl.block_table, 0, 1)
+    q = om.bf16_to_f64(wl.q[0, 0])
+    assert np.array_equal(O[0, 0], np.broadcast_to(C[0, :512], (4, 512)))
+    assert np.max(np.abs(L[0, 0] - SCALE * (q @ C[0]))) < 1e-12
+
+
+def test_zero_length_request():
+    wl = _tiny([0, 10], h=2)
+    O, L = oracle.decode(wl)
+    assert np.all(O[0] == 0) and np.all(np.isneginf(L[0]))
+
+
+@pytest.mark.parametrize("cuts", [[], [64], [1, 2, 3], [63, 64, 65, 300], list(range(64, 640, 64))])
+def test_split_combine_equals_unsplit(cuts):
+    # the split-KV merge (each piece's lse-weighted partial) reproduces the
+    # unsplit result: FlashMLA-2 newsletter, "Architectural Analysis"
+    wl = _tiny([700], h=3)
+    O, L = oracle.decode(wl)
+    edges = [0] + cuts + [700]
+    parts = [oracle.decode_chunk(wl, 0, 0, a, b) for a, b in zip(edges[:-1], edges[1:])]
+    Oc, Lc = oracle.combine(parts)
+    assert np.max(np.abs(Oc - O[0, 0])) < 1e-12 and np.max(np.abs(Lc - L[0, 0])) < 1e-12
+
+
+def test_causal_matches_masked_sdpa():
+    # the speculative step: query i sees keys j <= t - s + i; checked against
+    # the library attention with an explicit boolean mask
+    wl = _tiny([100, 64], h=3, s_q=5, causal=True)
+    O, L = oracle.decode(wl)
+    for r, t in enumerate(wl.seqlens):
+        t = int(t)
+        C = torch.from_numpy(om.gather_rows(wl.pool, wl.block_table, r, t))
+        Q = torch.from_numpy(om.bf16_to_f64(wl.q[r])).permute(1, 0, 2)          # h, s, 576
+        mask = torch.arange(t)[None, :] <= (t - 5 + torch.arange(5))[:, None]     # s, t
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q, C[None].expand(3, t, 576), C[None, :, :512].expand(3, t, 512), attn_mask=mask, scale=SCALE)
+        assert np.max(np.abs(O[r] - ref.permute(1, 0, 2).numpy())) < 1e-12
+
+
+def test_fp8_pages_dequantise_like_torch():
+    wl = _tiny([130], h=1, cache_dtype="fp8")
+    for pg in range(wl.num_pages):
+        rows = om.page_rows_f64(wl.pool, pg, wl.kv_scale)
+        raw = wl.pool[pg]
+        lat = raw[:64 * 512].view(torch.float8_e4m3fn).to(torch.float64).reshape(64, 512)
+        lat = lat * wl.kv_scale[pg].to(torch.float64)[:, None]
+        rope = raw[64 * 512:].view(torch.bfloat16).to(torch.float64).reshape(64, 64)
+        assert np.array_equal(rows[:, :512], lat.numpy())
+        assert np.array_equal(rows[:, 512:], rope.numpy())
+
+
+def test_nan_in_unused_slots_is_ignored():
+    wl = _tiny([70, 10], h=2)
+    O, L = oracle.decode(wl)
+    # poison every slot past each request's length and every unreferenced page
+    used = set()
+    for r, t in enumerate(wl.seqlens):
+        n = (int(t) + 63) // 64
+        used |= set(int(x) for x in wl.block_table[r, :n])
+        last = int(wl.block_table[r, n - 1])
+        if t % 64:
+            wl.pool[last, int(t) % 64:] = float("nan")
+    extra = mw.make(1, 1, 1, [64], seed=9).pool.fill_(float("nan"))
+    wl.pool = torch.cat([wl.pool, extra])
+    O2, L2 = oracle.decode(wl)
+    assert np.isfinite(O2).all() and np.array_equal(O, O2) and np.array_equal(L, L2)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each must trip at least one pin above
+# --------------------------------------------------------------------------
+
+def _attend_no_rope(qrows, C, scale):
+    return om.attend(np.concatenate([qrows[:, :512], np.zeros_like(qrows[:, 512:])], 1), C, scale)
+
+
+def _attend_wrong_scale(qrows, C, scale):
+    return om.attend(qrows, C, 1.0 / math.sqrt(576.0))
+
+
+def _attend_values_from_tail(qrows, C, scale):
+    O, L = om.attend(qrows, C, scale)
+    x = scale * (qrows @ C.T)
+    w = np.exp(x - L[:, None])
+    return w @ C[:, 64:], L
+
+
+def _attend_transposed(qrows, C, scale):
+    O, L = om.attend(qrows, C, scale)
+    return O[:, ::-1].copy(), L
+
+
+@pytest.mark.parametrize("bad", [_attend_no_rope, _attend_wrong_scale, _attend_values_from_tail,
+                                 _attend_transposed])
+def test_planted_mistakes_are_caught(bad):
+    case = _absorption_case(seed=5)
+    ref = _mha_reference(*case).numpy()
+    got = _latent_path(bad, *case)
+    assert np.max(np.abs(got - ref)) > 1e-3
+
+
+def test_planted_page_index_mistake_is_caught(monkeypatch):
+    # a wrong block-table lookup in the vectorised oracle must disagree with
+    # the brute-force loop, which reads the table on its own
+    wl = _tiny([130], h=2)
+    Ob, _ = oracle.brute(wl)
+    orig = om.gather_rows
+
+    def wrong_page(pool, table, r, n, kv_scale=None, start=0):
+        return orig(pool, np.roll(np.asarray(table), 1, axis=1), r, n, kv_scale, start)
+    monkeypatch.setattr(om, "gather_rows", wrong_page)
+    O2, _ = om.decode(wl)
+    assert np.max(np.abs(O2 - Ob)) > 1e-3
