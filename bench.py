@@ -1,0 +1,342 @@
+#!/usr/bin/env python
+"""Benchmark of MLA decode in absorbed latent space on B200.
+
+One step = one pass of the whole decode path over one batch: the split-KV
+schedule, the decode kernel and the combine kernel, all through the C ABI
+(libmla_b200.so).  The workload is the DeepSeek-V3-shaped decode batch
+(b=64, s_q=1, h=128, k=512, p=64, t=4096, 64-token pages, random block
+table), synthetic bf16 N(0,1) data.  The metric is TFLOP/s by the page's
+cost model (FLOPs = 2 b h s t (2k+p)); the KV GB/s by the same model is
+reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs an independent replica on its own GPU (the
+requests shard with no exchange step); the whole-job value sums all ranks'
+FLOPs over the slowest rank's time.  `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_workloads as mw  # noqa: E402
+from mla_workloads import cost  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & KV GB/s vs B200 roofline (h=128,k=512,p=64,t=4096)"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out = self.proc.communicate(timeout=5)[0]
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out = self.proc.communicate()[0]
+        sms, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sms),
+                "power_w_max": max(power) if power else None}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(wl, n_req):
+    """Times the fp64 oracle on the first n_req requests; returns
+    (seconds, flops of the sample, description)."""
+    import oracle
+    rows = [(r, i) for r in range(n_req) for i in range(wl.s_q)]
+    t0 = time.perf_counter()
+    oracle.decode(wl, rows=rows)
+    dt = time.perf_counter() - t0
+    st = int(wl.seqlens[:n_req].astype(np.int64).sum())
+    fl = cost.mla_flops(n_req, wl.num_heads, wl.s_q, None, sum_t=st)
+    return dt, fl, f"{n_req} of {wl.batch} requests ({st} cached tokens, all {wl.num_heads} heads)"
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    n_req = max(1, min(wl.batch, args.ref_requests))
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(wl, 1)   # warm the BLAS threads (untimed)
+    times, fl, desc = [], 0.0, ""
+    for _ in range(args.steps):
+        dt, fl, desc = oracle_sample(wl, n_req)
+        times.append(dt)
+    sec = sum(times) / len(times)
+    tflops = fl / sec / 1e12
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.num_heads,
+                       "seq_len": int(wl.seqlens.max()), "sample": desc},
+            "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl, world, rank, local):
+    import mla_latent_space_b200 as mla
+    from mla_latent_space_b200 import build
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages, wl.cache_dtype, wl.causal)
+    q = wl.q.to(dev)
+    pool = wl.pool.to(dev)
+    kv_scale = None if wl.kv_scale is None else wl.kv_scale.to(dev)
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    sl = torch.from_numpy(wl.seqlens).to(dev)
+    out = torch.empty((wl.batch, wl.s_q, wl.num_heads, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.s_q, wl.num_heads), dtype=torch.float32, device=dev)
+    dec = mla.Decoder(shape, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    decode_fn = mla.mla_decode_fwd_simt if args.simt else mla.mla_decode_fwd
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        dec.schedule(sl)
+        if ev is not None:
+            ev[0].record(stream)
+        decode_fn(shape, q, pool, kv_scale, bt, sl, wl.softmax_scale, dec.sched, dec.workspace, out, lse)
+        if ev is not None:
+            ev[1].record(stream)
+        mla.mla_combine(shape, dec.sched, dec.workspace, out, lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {mla.error_string(st)}")
+
+    K = args.steps
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()                       # L2 flush outside the timed events
+        ev_step[k][0].record(stream)
+        step(ev_dec[k])
+        ev_step[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    my_ms = sum(step_ms) / K
+    ms = max_over_ranks(my_ms, world)
+    dec_avg_ms = sum(dec_ms) / K
+    st = dec.status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {mla.error_string(st)}")
+
+    # end to end through the public API with host buffers: per step the
+    # query, block table and lengths go host->device, the output and lse
+    # come back device->host (the KV cache is resident device state)
+    h_q = wl.q.pin_memory()
+    h_bt = torch.from_numpy(wl.block_table).pin_memory()
+    h_sl = torch.from_numpy(wl.seqlens).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = h_q.numel() * 2 + h_bt.numel() * 4 + h_sl.numel() * 4
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        sl.copy_(h_sl, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev_e2e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world)
+    for k in range(K):
+        flush.zero_()
+        ev_e2e[k][0].record(stream)
+        e2e_step()
+        ev_e2e[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev_e2e) / K, world)
+
+    flops, nbytes = cost.workload_cost(wl)
+    pk, pk_kind = peaks()
+    value = world * flops / (ms * 1e-3) / 1e12
+    dec_gbs = nbytes / (dec_avg_ms * 1e-3) / 1e9
+    dec_tflops = flops / (dec_avg_ms * 1e-3) / 1e12
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": dec_gbs / pk["hbm_gbs"], "traffic": args.traffic}
+    else:
+        roof = {"bound": "tensor", "achieved": dec_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": dec_tflops / pk["bf16_tflops"], "traffic": args.traffic}
+    roof["kernel"] = "mla_decode_fwd (simt debug path)" if args.simt else "mla_decode_fwd"
+    roof["peak_kind"] = f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback"
+    roof["launch_us"] = dec_avg_ms * 1e3
+    roof["tensor_frac"] = dec_tflops / pk["bf16_tflops"]
+    roof["tensor_frac_sustained"] = dec_tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.num_heads,
+                       "seq_len": int(wl.seqlens.max()), "sum_t": wl.total_tokens, "page": 64,
+                       "cache": wl.cache_dtype, "parallelism": f"replicas x{world}",
+                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+            "kv_gbs": world * nbytes / (ms * 1e-3) / 1e9,
+            "us_per_step": ms * 1e3,
+            "roofline": roof,
+            "clocks": clk,
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * K}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # about 10 s of oracle work: the sample repeated until 10 s have passed
+        n_req = max(1, min(wl.batch, args.ref_requests))
+        tot_dt, tot_fl, reps = 0.0, 0.0, 0
+        while tot_dt < 10.0 and reps < 50:
+            dt, fl, desc = oracle_sample(wl, n_req)
+            tot_dt, tot_fl, reps = tot_dt + dt, tot_fl + fl, reps + 1
+        line["cpu_baseline"] = {"value": tot_fl / tot_dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": f"{desc}, x{reps}", "seconds": tot_dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2, help="workload 1-5 (2 = the headline decode batch)")
+    ap.add_argument("--simt", action="store_true", help="time the SIMT debug kernel instead")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per decode launch for the current kernel (else null)")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args.gpus)
+    wl = mw.make_config(args.config, seed=0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, world, rank)
+        else:
+            run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

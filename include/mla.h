@@ -1,0 +1,170 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA decode library, libmla_b200.so.
+ *
+ * Multi-head Latent Attention decode in absorbed latent space ("MLA Cost
+ * Analysis & Regime Guide", section "Absorption Trick"): with the key and
+ * value up-projections absorbed into the query and the output projection,
+ * every head scores directly against the shared latent cache,
+ *
+ *     S = scale * Qz . C^T            C = cache rows [latent 512 | RoPE 64]
+ *     O = softmax(S) . C[:, :512]     (decompression O . W_v^T is left to a
+ *                                      separate GEMM, outside this library)
+ *
+ * Shapes follow the page's "Tensor Shapes" table (h=128, k=512, p=64).  The
+ * split-KV scheduler and the log-sum-exp merge of partial results follow the
+ * FlashMLA-2 newsletter page ("Architectural Analysis": sequence partitions
+ * balanced across SMs for jagged batches).
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library never allocates device memory, never frees caller memory and
+ *    never synchronises the stream (except mla_get_device_status, which
+ *    says so).
+ *  - Every call takes the caller's cudaStream_t (passed as void*: NULL is
+ *    the legacy default stream) and enqueues its work there.
+ *  - Return value: MLA_OK (0) or a negative MLA_ERR_* code.  Arguments are
+ *    validated on the host BEFORE anything is launched; an error return
+ *    means nothing was enqueued.  mla_error_string() names each code.
+ *  - Layouts are dense and row-major (innermost dimension last, contiguous).
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes --------------------------------------------------------- */
+enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer      */
+  MLA_ERR_UNSUPPORTED = -2,  /* shape the kernels do not implement             */
+  MLA_ERR_WORKSPACE = -3,    /* workspace / schedule buffer too small          */
+  MLA_ERR_CUDA = -4,         /* a CUDA runtime call failed (launch, attribute) */
+  MLA_ERR_TIMEOUT = -5,      /* device status: a bounded wait gave up          */
+  MLA_ERR_DEVICE_CHECK = -6  /* device status: seqlen / page id out of range   */
+};
+
+/* ---- cache element types -------------------------------------------------- */
+enum {
+  MLA_CACHE_BF16 = 0,      /* page = 64 rows x 576 bf16 = 73,728 bytes           */
+  MLA_CACHE_FP8_E4M3 = 1   /* page = 64x512 e4m3 bytes, then 64x64 bf16 RoPE
+                              values (40,960 bytes); scales in kv_scale       */
+};
+
+/* Fixed geometry of this library (DeepSeek-V3 defaults of the page's
+ * "Tensor Shapes" table; one 128-row tile = 128 (query token, head) rows). */
+#define MLA_D_QK 576
+#define MLA_D_V 512
+#define MLA_PAGE_SIZE 64
+#define MLA_TILE_ROWS 128
+
+/* Problem description.  Every field is read on the host only. */
+typedef struct {
+  int32_t batch;             /* b: requests in the batch, >= 1                  */
+  int32_t s_q;               /* query tokens per request (1 = decode, >1 = spec) */
+  int32_t num_heads;         /* h: query heads; s_q*h rows are tiled by 128    */
+  int32_t d_qk;              /* must be 576 (k + p)                             */
+  int32_t d_v;               /* must be 512 (k)                                 */
+  int32_t page_size;         /* must be 64                                      */
+  int32_t max_pages_per_seq; /* row length of block_table, >= 1                 */
+  int32_t num_pages;         /* pages in the cache pool, >= 1                   */
+  int32_t cache_dtype;       /* MLA_CACHE_BF16 or MLA_CACHE_FP8_E4M3            */
+  int32_t causal;            /* 1: query token i sees keys j <= t - s_q + i    */
+} mla_shape_t;
+
+/* Bytes of the device buffer mla_get_schedule fills.  num_sms is the SM
+ * count of the device that will run the decode (one scheduler worker per
+ * pair of SMs).  Returns 0 for an invalid shape. */
+size_t mla_schedule_bytes(const mla_shape_t* shape, int num_sms);
+
+/* Bytes of the device workspace mla_decode_fwd / mla_combine use: fp32
+ * partial results of split tiles (at most 2 per worker, 128x512 O + 128
+ * lse each) plus a 256-byte status area.  Returns 0 for an invalid shape. */
+size_t mla_workspace_bytes(const mla_shape_t* shape, int num_sms);
+
+/* a1 -- split-KV schedule (FlashMLA-2 newsletter, "Architectural Analysis").
+ * Splits the work sum over tiles of (visible pages + a fixed per-piece
+ * cost) into num_sms/2 contiguous, equally costed ranges of (tile, page)
+ * units, and records for every tile how many pieces it was cut into and
+ * where their partial results go.  Runs one small kernel on `stream`.
+ *   seqlens : device int32 [batch], tokens in the cache per request
+ *             INCLUDING the s_q new ones.  Values outside
+ *             [0, max_pages_per_seq*64] are clamped and flagged
+ *             (MLA_ERR_DEVICE_CHECK from mla_get_device_status).
+ *   sched   : device buffer of mla_schedule_bytes(shape, num_sms) bytes,
+ *             4-byte aligned; written entirely by this call.
+ * The schedule depends only on seqlens, so one schedule serves every layer
+ * of a decode step. */
+int mla_get_schedule(const mla_shape_t* shape, const int32_t* seqlens, int num_sms,
+                     void* sched, size_t sched_bytes, void* stream);
+
+/* a2-a7 (+a9 FP8, a10 causal) -- the decode itself.
+ *   q          : bf16 [batch, s_q, num_heads, 576], the absorbed query rows
+ *                (q_nope . W_k ++ q_pe), 16-byte aligned.
+ *   kv_cache   : page pool.  BF16: bf16 [num_pages, 64, 576].  FP8: uint8
+ *                [num_pages, 40960] (64x512 e4m3 then 64x64 bf16 RoPE).
+ *                1024-byte aligned base.  Value rows are the first 512
+ *                entries of each cache row.
+ *   kv_scale   : FP8 only: fp32 [num_pages, 64], one dequantisation scale
+ *                per cached token (value = e4m3 * scale).  NULL for BF16.
+ *   block_table: int32 [batch, max_pages_per_seq]; entry [r][j] is the pool
+ *                page holding tokens 64j..64j+63 of request r.  Entries past
+ *                ceil(visible/64) are never read.  Out-of-range page ids are
+ *                skipped and flagged (MLA_ERR_DEVICE_CHECK).
+ *   seqlens    : the same int32 [batch] array given to mla_get_schedule.
+ *   softmax_scale : multiplies the raw 576-d dot product before softmax.
+ *   sched      : filled by mla_get_schedule for this shape and num_sms.
+ *   workspace  : mla_workspace_bytes(shape, num_sms) bytes, 256-byte
+ *                aligned; the caller must not touch it between this call and
+ *                mla_combine.
+ *   out        : bf16 [batch, s_q, num_heads, 512], the latent output rows.
+ *   lse        : fp32 [batch, s_q, num_heads], natural-log log-sum-exp of the
+ *                scaled scores (-inf for a row that sees no key).
+ * Tiles cut into several pieces are finished by mla_combine; tiles in one
+ * piece are written directly.  Call mla_combine after every decode. */
+int mla_decode_fwd(const mla_shape_t* shape, const void* q, const void* kv_cache,
+                   const float* kv_scale, const int32_t* block_table, const int32_t* seqlens,
+                   float softmax_scale, const void* sched, void* workspace, size_t workspace_bytes,
+                   void* out, float* lse, void* stream);
+
+/* a8 -- log-sum-exp merge of split pieces: for each split row,
+ * L = ln sum_i e^{lse_i}, O = sum_i e^{lse_i - L} O_i; writes out/lse for
+ * split tiles and for tiles that see no key at all (O = 0, lse = -inf).
+ * Arguments as for mla_decode_fwd. */
+int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace,
+                size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/* Debug path, used by the tests only: the same decode computed by a plain
+ * SIMT kernel (fp32 FMA, no tensor cores) over the same schedule and
+ * workspace.  Never chosen by mla_decode_fwd. */
+int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_cache,
+                        const float* kv_scale, const int32_t* block_table,
+                        const int32_t* seqlens, float softmax_scale, const void* sched,
+                        void* workspace, size_t workspace_bytes, void* out, float* lse,
+                        void* stream);
+
+/* Reads and clears the sticky device status words that the scheduler and
+ * the decode kernels set instead of trapping (a bounded wait that gave up,
+ * an out-of-range seqlen or page id).  SYNCHRONISES `stream`.  *status
+ * receives MLA_OK, MLA_ERR_TIMEOUT or MLA_ERR_DEVICE_CHECK. */
+int mla_get_device_status(const void* sched, void* workspace, void* stream, int* status);
+
+/* Host copy of the scheduler (same code as the device kernel), for tests
+ * and tools: seqlens and sched are HOST pointers here. */
+int mla_plan_schedule_host(const mla_shape_t* shape, const int32_t* seqlens, int num_sms,
+                           void* sched, size_t sched_bytes);
+
+/* Human-readable name of an MLA_* code (static storage). */
+const char* mla_error_string(int code);
+
+/* Library version string (static storage). */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H */

@@ -1,0 +1,212 @@
+// Host side of libmla_b200.so: argument validation, buffer sizing and the
+// launches behind the C ABI declared in include/mla.h.  Every check runs
+// before anything is enqueued; an error return means the stream is untouched.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace mla {
+void plan_schedule_host(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched);
+cudaError_t launch_schedule(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched, cudaStream_t st);
+cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_scale, const int32_t* block_table,
+                               const int32_t* seqlens, float scale, const void* sched, void* ws, void* out,
+                               float* lse, int num_pages, int fp8, int cap_slots, int grid_ctas,
+                               cudaStream_t stream);
+cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
+                           int cap_slots, cudaStream_t stream);
+int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
+                        const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
+                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
+}  // namespace mla
+
+using namespace mla;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every entry point.
+int check_shape(const mla_shape_t* s) {
+  if (!s) return MLA_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->s_q < 1 || s->num_heads < 1 || s->max_pages_per_seq < 1 || s->num_pages < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (s->d_qk != MLA_D_QK || s->d_v != MLA_D_V || s->page_size != MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED;
+  if (s->cache_dtype != MLA_CACHE_BF16 && s->cache_dtype != MLA_CACHE_FP8_E4M3) return MLA_ERR_UNSUPPORTED;
+  if (s->causal != 0 && s->causal != 1) return MLA_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(s->s_q) * s->num_heads;
+  const int64_t tiles = int64_t(s->batch) * ((rows + MLA_TILE_ROWS - 1) / MLA_TILE_ROWS);
+  if (rows * s->batch >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED;
+  if (int64_t(s->max_pages_per_seq) * MLA_PAGE_SIZE >= (int64_t(1) << 30)) return MLA_ERR_UNSUPPORTED;
+  if (tiles * (int64_t(s->max_pages_per_seq) + kPieceOverhead) >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+ShapeInfo shape_info(const mla_shape_t* s) {
+  ShapeInfo si;
+  si.batch = s->batch;
+  si.s_q = s->s_q;
+  si.heads = s->num_heads;
+  si.causal = s->causal;
+  si.max_pages = s->max_pages_per_seq;
+  si.tiles_per_req = (s->s_q * s->num_heads + MLA_TILE_ROWS - 1) / MLA_TILE_ROWS;
+  return si;
+}
+
+size_t sched_bytes_for(const mla_shape_t* s, int num_sms) {
+  ShapeInfo si = shape_info(s);
+  int W = num_workers_for(num_sms);
+  return 4 * (size_t(kHeaderInts) + size_t(W) * kWorkerInts + size_t(si.batch) * si.tiles_per_req * kTileInts);
+}
+
+int cap_slots_for(size_t ws_bytes) {
+  if (ws_bytes < kStatusBytes) return -1;
+  size_t cap = (ws_bytes - kStatusBytes) / kSlotBytes;
+  return cap > (1u << 30) ? (1 << 30) : int(cap);
+}
+
+int device_sms(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  static std::mutex mu;
+  static int cache[64] = {0};
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return MLA_ERR_CUDA;
+    cache[dev] = n;
+  }
+  *out = cache[dev];
+  return MLA_OK;
+}
+
+int check_decode_args(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
+                      const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
+                      void* ws, size_t ws_bytes, void* out, float* lse) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  if (!q || !kv || !block_table || !seqlens || !sched || !ws || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (shape->cache_dtype == MLA_CACHE_FP8_E4M3 && !kv_scale) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv, 256) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(block_table, 4) ||
+      !aligned(seqlens, 4) || !aligned(sched, 16) || !aligned(ws, 256) || (kv_scale && !aligned(kv_scale, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
+  if (cap_slots_for(ws_bytes) < 0) return MLA_ERR_WORKSPACE;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mla_schedule_bytes(const mla_shape_t* shape, int num_sms) {
+  if (check_shape(shape) != MLA_OK || num_sms < 1) return 0;
+  return sched_bytes_for(shape, num_sms);
+}
+
+size_t mla_workspace_bytes(const mla_shape_t* shape, int num_sms) {
+  if (check_shape(shape) != MLA_OK || num_sms < 1) return 0;
+  return kStatusBytes + size_t(max_slots_for(num_workers_for(num_sms))) * kSlotBytes;
+}
+
+int mla_get_schedule(const mla_shape_t* shape, const int32_t* seqlens, int num_sms, void* sched,
+                     size_t sched_bytes, void* stream) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  if (!seqlens || !sched || num_sms < 1) return MLA_ERR_INVALID_ARG;
+  if (!aligned(sched, 16) || !aligned(seqlens, 4)) return MLA_ERR_INVALID_ARG;
+  if (sched_bytes < sched_bytes_for(shape, num_sms)) return MLA_ERR_WORKSPACE;
+  cudaError_t e = launch_schedule(seqlens, shape_info(shape), num_workers_for(num_sms), static_cast<int32_t*>(sched),
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_plan_schedule_host(const mla_shape_t* shape, const int32_t* seqlens, int num_sms, void* sched,
+                           size_t sched_bytes) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  if (!seqlens || !sched || num_sms < 1) return MLA_ERR_INVALID_ARG;
+  if (sched_bytes < sched_bytes_for(shape, num_sms)) return MLA_ERR_WORKSPACE;
+  plan_schedule_host(seqlens, shape_info(shape), num_workers_for(num_sms), static_cast<int32_t*>(sched));
+  return MLA_OK;
+}
+
+int mla_decode_fwd(const mla_shape_t* shape, const void* q, const void* kv_cache, const float* kv_scale,
+                   const int32_t* block_table, const int32_t* seqlens, float softmax_scale, const void* sched,
+                   void* workspace, size_t workspace_bytes, void* out, float* lse, void* stream) {
+  int rc = check_decode_args(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                             workspace_bytes, out, lse);
+  if (rc != MLA_OK) return rc;
+  return launch_decode_sm100(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                             cap_slots_for(workspace_bytes), out, lse, static_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_cache, const float* kv_scale,
+                        const int32_t* block_table, const int32_t* seqlens, float softmax_scale,
+                        const void* sched, void* workspace, size_t workspace_bytes, void* out, float* lse,
+                        void* stream) {
+  int rc = check_decode_args(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                             workspace_bytes, out, lse);
+  if (rc != MLA_OK) return rc;
+  int sms = 0;
+  if ((rc = device_sms(&sms)) != MLA_OK) return rc;
+  cudaError_t e = launch_decode_simt(q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                                     out, lse, shape->num_pages, shape->cache_dtype == MLA_CACHE_FP8_E4M3,
+                                     cap_slots_for(workspace_bytes), sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace, size_t workspace_bytes,
+                void* out, float* lse, void* stream) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  if (!sched || !workspace || !out || !lse) return MLA_ERR_INVALID_ARG;
+  if (!aligned(sched, 16) || !aligned(workspace, 256) || !aligned(out, 16) || !aligned(lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  const int cap = cap_slots_for(workspace_bytes);
+  if (cap < 0) return MLA_ERR_WORKSPACE;
+  ShapeInfo si = shape_info(shape);
+  cudaError_t e = launch_combine(sched, workspace, out, lse, si.batch * si.tiles_per_req, cap,
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_get_device_status(const void* sched, void* workspace, void* stream, int* status) {
+  if (!sched || !workspace || !status) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t ws_word = 0, sched_word = 0;
+  if (cudaMemcpyAsync(&ws_word, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyAsync(&sched_word, static_cast<const int32_t*>(sched) + H_STATUS, 4, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MLA_ERR_CUDA;
+  const int32_t all = ws_word | sched_word;
+  if (all & kStatusTimeout) *status = MLA_ERR_TIMEOUT;
+  else if (all & kStatusWorkspace) *status = MLA_ERR_WORKSPACE;
+  else if (all) *status = MLA_ERR_DEVICE_CHECK;
+  else *status = MLA_OK;
+  return MLA_OK;
+}
+
+const char* mla_error_string(int code) {
+  switch (code) {
+    case MLA_OK: return "MLA_OK: success";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: null pointer, bad size or misaligned pointer";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: shape not implemented (d_qk 576, d_v 512, page 64)";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: schedule or workspace buffer too small";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device wait gave up";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: out-of-range seqlen or page id seen on the device";
+    default: return "MLA: unknown error code";
+  }
+}
+
+const char* mla_version(void) { return "mla_b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

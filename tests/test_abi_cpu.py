@@ -1,0 +1,214 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+function include/mla.h declares, sizes its buffers, and rejects bad
+arguments before launching anything.  The scheduler's host copy (the same
+code as the device kernel) is checked for exact coverage and balance."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_space_b200 as mla
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    from mla_latent_space_b200 import build
+    build.build()
+    L = mla.lib()
+    names = _declared()
+    assert "mla_decode_fwd" in names and "mla_get_schedule" in names and "mla_combine" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(mla.EXPORTED) <= set(names)
+    assert b"sm_100a" in L.mla_version()
+
+
+def test_error_strings():
+    for code in range(0, -7, -1):
+        s = mla.error_string(code)
+        assert s.startswith("MLA_")
+    assert "unknown" in mla.error_string(42)
+
+
+def _shape(**kw):
+    base = dict(batch=2, s_q=1, num_heads=128, max_pages_per_seq=4, num_pages=8)
+    base.update(kw)
+    return mla.make_shape(**base)
+
+
+def test_buffer_sizes():
+    s = _shape()
+    # header 16 + 74 workers x 8 + 2 tiles x 4 int32 words
+    assert mla.mla_schedule_bytes(s, 148) == 4 * (16 + 74 * 8 + 2 * 4)
+    assert mla.mla_workspace_bytes(s, 148) == 256 + 148 * (128 * 512 * 4 + 128 * 4)
+    s5 = _shape(batch=32, s_q=16, num_heads=128, max_pages_per_seq=64)
+    assert mla.mla_schedule_bytes(s5, 148) == 4 * (16 + 74 * 8 + 32 * 16 * 4)
+    bad = _shape()
+    bad.d_qk = 192
+    assert mla.mla_schedule_bytes(bad, 148) == 0
+
+
+def _call_decode(shape, **over):
+    fake = ctypes.c_void_p(1 << 20)     # never dereferenced: validation fails first
+    args = dict(q=fake, kv=fake, kv_scale=None, bt=fake, sl=fake, scale=0.07, sched=fake, ws=fake,
+                ws_bytes=1 << 20, out=fake, lse=fake)
+    args.update(over)
+    return mla.lib().mla_decode_fwd(ctypes.byref(shape), args["q"], args["kv"], args["kv_scale"], args["bt"],
+                                    args["sl"], args["scale"], args["sched"], args["ws"], args["ws_bytes"],
+                                    args["out"], args["lse"], None)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d_qk", 192, -2), ("d_v", 128, -2), ("page_size", 16, -2), ("cache_dtype", 7, -2),
+    ("batch", 0, -1), ("s_q", 0, -1), ("num_heads", 0, -1), ("max_pages_per_seq", 0, -1),
+    ("num_pages", 0, -1), ("causal", 2, -1)])
+def test_decode_rejects_bad_shapes(field, value, code):
+    s = _shape()
+    setattr(s, field, value)
+    assert _call_decode(s) == code
+
+
+def test_decode_rejects_bad_pointers():
+    s = _shape()
+    assert _call_decode(s, q=None) == -1
+    assert _call_decode(s, out=None) == -1
+    assert _call_decode(s, q=ctypes.c_void_p((1 << 20) + 2)) == -1          # q not 16-byte aligned
+    assert _call_decode(s, kv=ctypes.c_void_p((1 << 20) + 64)) == -1        # pool not 256-byte aligned
+    assert _call_decode(s, ws=ctypes.c_void_p((1 << 20) + 16)) == -1
+    assert _call_decode(s, scale=float("nan")) == -1
+    assert _call_decode(s, ws_bytes=16) == -3
+    s8 = _shape(cache_dtype="fp8")
+    assert _call_decode(s8, kv_scale=None) == -1                             # fp8 needs scales
+
+
+def test_schedule_and_combine_reject_bad_args():
+    s = _shape()
+    fake = ctypes.c_void_p(1 << 20)
+    L = mla.lib()
+    assert L.mla_get_schedule(ctypes.byref(s), None, 148, fake, 1 << 20, None) == -1
+    assert L.mla_get_schedule(ctypes.byref(s), fake, 148, fake, 16, None) == -3
+    assert L.mla_get_schedule(ctypes.byref(s), fake, 0, fake, 1 << 20, None) == -1
+    assert L.mla_combine(ctypes.byref(s), None, fake, 1 << 20, fake, fake, None) == -1
+    assert L.mla_combine(ctypes.byref(s), fake, fake, 8, fake, fake, None) == -3
+    assert L.mla_get_device_status(None, fake, None, None) == -1
+
+
+# --------------------------------------------------------------------------
+# host scheduler
+# --------------------------------------------------------------------------
+
+def parse_schedule(buf, shape):
+    a = buf.numpy().astype(np.int64)
+    W, T = int(a[1]), int(a[2])
+    workers = a[16:16 + 8 * W].reshape(W, 8)
+    tiles = a[16 + 8 * W:16 + 8 * W + 4 * T].reshape(T, 4)
+    return dict(hdr=a[:16], W=W, T=T, workers=workers, tiles=tiles)
+
+
+def pieces_of(sc):
+    """Expand worker ranges into (worker, tile, p0, p1, split) pieces."""
+    out = []
+    for w, (tb, pb, te, pe, fs, *_r) in enumerate(sc["workers"]):
+        T = tb
+        while T <= te and T < sc["T"]:
+            pages = sc["tiles"][T, 0]
+            p0 = pb if T == tb else 0
+            p1 = pe if T == te else pages
+            p1 = min(p1, pages)
+            if p0 < p1:
+                out.append((w, T, p0, p1, fs if T == tb else 0))
+            T += 1
+    return out
+
+
+def check_schedule(seqlens, s_q, h, causal, n_sms):
+    b = len(seqlens)
+    maxp = max(1, (max(seqlens) + 63) // 64)
+    shape = mla.make_shape(b, s_q, h, maxp, 1, causal=causal)
+    sc = parse_schedule(mla.mla_plan_schedule_host(shape, torch.tensor(seqlens, dtype=torch.int32), n_sms), shape)
+    W = max(1, n_sms // 2)
+    tpr = (s_q * h + 127) // 128
+    assert sc["W"] == W and sc["T"] == b * tpr
+    # visible pages per tile (the rows of a tile are (query token, head) pairs)
+    for T in range(b * tpr):
+        r, qt = divmod(T, tpr)
+        last_row = min(s_q * h, 128 * (qt + 1)) - 1
+        i = last_row // h
+        L = seqlens[r] - s_q + i + 1 if causal else seqlens[r]
+        assert sc["tiles"][T, 0] == (max(L, 0) + 63) // 64
+    pcs = pieces_of(sc)
+    # every (tile, page) unit exactly once
+    cover = {}
+    for w, T, p0, p1, split in pcs:
+        for p in range(p0, p1):
+            assert (T, p) not in cover
+            cover[(T, p)] = w
+    want = {(T, p) for T in range(b * tpr) for p in range(sc["tiles"][T, 0])}
+    assert set(cover) == want
+    # split bookkeeping: pieces of a tile are numbered 0..n-1 in order and
+    # their slots are disjoint and within 2W
+    slots = set()
+    by_tile = {}
+    for w, T, p0, p1, split in pcs:
+        by_tile.setdefault(T, []).append((p0, split))
+    for T, lst in by_tile.items():
+        n = sc["tiles"][T, 2]
+        assert n == len(lst)
+        assert [s for _, s in sorted(lst)] == list(range(n))
+        if n > 1:
+            for k in range(n):
+                slot = sc["tiles"][T, 3] + k
+                assert slot not in slots
+                slots.add(slot)
+    assert len(slots) <= 2 * W and sc["hdr"][5] == len(slots)
+    for T in range(b * tpr):
+        if sc["tiles"][T, 0] == 0:
+            assert sc["tiles"][T, 2] == 0
+    # balance: no worker exceeds the even share by more than one piece's overhead + 1 page
+    cost = np.zeros(W)
+    for w, T, p0, p1, split in pcs:
+        cost[w] += (p1 - p0) + 2
+    total = sc["hdr"][4]
+    assert cost.max() <= total / W + 2 * 2 + 1
+    return sc
+
+
+@pytest.mark.parametrize("n_sms", [2, 3, 8, 148, 300])
+def test_schedule_uniform(n_sms):
+    check_schedule([4096] * 64, 1, 128, False, n_sms)
+
+
+def test_schedule_jagged_and_special_lengths():
+    import mla_workloads as mw
+    _, _, _, lens = mw.config_shape(3)
+    sc = check_schedule(list(lens), 1, 128, False, 148)
+    # the forced 131072-token request is cut into several pieces
+    r = int(np.argmax(lens))
+    assert sc["tiles"][r, 2] > 1
+    check_schedule([0, 1, 63, 64, 65, 0, 128, 5000], 1, 16, False, 148)
+    check_schedule([0, 0, 0], 1, 128, False, 148)
+
+
+def test_schedule_spec_causal_and_packed_rows():
+    check_schedule([4096] * 32, 16, 128, True, 148)
+    check_schedule([5, 17, 16, 100], 16, 16, True, 20)   # 2 query tokens per 128-row tile
+    check_schedule([3, 200], 4, 48, True, 10)             # tiles straddle query tokens
+
+
+def test_schedule_clamps_bad_lengths():
+    shape = mla.make_shape(3, 1, 128, 2, 1)
+    buf = mla.mla_plan_schedule_host(shape, torch.tensor([-5, 1000, 64], dtype=torch.int32), 8)
+    sc = parse_schedule(buf, shape)
+    assert sc["hdr"][6] != 0                       # status flags the clamp
+    assert list(sc["tiles"][:, 0]) == [0, 2, 1]

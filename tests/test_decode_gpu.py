@@ -1,0 +1,103 @@
+"""GPU parity of the decode path (schedule -> decode -> combine through the
+C ABI) against the fp64 oracle, on the five workloads and their edge cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mla_latent_space_b200 as mla
+import mla_workloads as mw
+import oracle
+from gpu_helpers import (assert_parity, check_full, check_sampled, compare, run, shape_of, to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mla_latent_space_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+# ---- small cases the oracle finishes in seconds ---------------------------
+
+def test_config1_tiny_full():
+    check_full(mw.make_config(1))
+
+
+@pytest.mark.parametrize("lens", [[1], [63, 64, 65], [700, 1, 129, 4096], [0, 77]])
+def test_ragged_lengths_h128(lens):
+    check_full(mw.make(len(lens), 1, 128, lens, seed=11, name=f"ragged{lens}"))
+
+
+def test_small_jagged_h128():
+    check_full(mw.make(6, 1, 128, None, jagged=(128, 3000), seed=4, name="jagged_small"))
+
+
+def test_small_fp8():
+    check_full(mw.make(3, 1, 128, [300, 64, 1000], cache_dtype="fp8", seed=5, name="fp8_small"))
+
+
+def test_small_causal_spec():
+    check_full(mw.make(3, 16, 128, [200, 16, 700], causal=True, seed=6, name="spec_small"))
+
+
+@pytest.mark.parametrize("h,s_q,causal", [(16, 1, False), (64, 2, True), (48, 4, True), (128, 2, False)])
+def test_head_counts_and_packed_tiles(h, s_q, causal):
+    check_full(mw.make(3, s_q, h, [130, 5, 260], causal=causal, seed=7, name=f"h{h}s{s_q}"))
+
+
+def test_simt_debug_path_matches_oracle():
+    check_full(mw.make(3, 1, 128, [300, 64, 1000], seed=8), simt=True)
+    check_full(mw.make(2, 16, 128, [100, 300], causal=True, seed=8), simt=True)
+
+
+@pytest.mark.parametrize("n_sms", [2, 16, 148, 1000])
+def test_split_counts_agree(n_sms):
+    # the same rows, cut into 1 .. hundreds of pieces, stay within tolerance
+    wl = mw.make(4, 1, 128, [3000, 64, 1, 2500], seed=9, name="splits")
+    check_full(wl, n_sms=n_sms)
+
+
+def test_nan_in_unused_slots_and_pages():
+    wl = mw.make(3, 1, 128, [70, 130, 1], seed=10, name="poison")
+    O0, L0, _ = run(wl)
+    for r, t in enumerate(wl.seqlens):
+        n = (int(t) + 63) // 64
+        last = int(wl.block_table[r, n - 1])
+        if t % 64:
+            wl.pool[last, int(t) % 64:] = float("nan")
+        wl.block_table[r, n:] = 0
+    extra = torch.full((2, 64, 576), float("nan"), dtype=torch.bfloat16)
+    wl.pool = torch.cat([wl.pool, extra])
+    O1, L1, st = run(wl)
+    assert st == 0 and np.isfinite(O1).all() and np.array_equal(O0, O1) and np.array_equal(L0, L1)
+
+
+def test_device_schedule_equals_host_planner():
+    import mla_workloads as mw2
+    for cfg in (2, 3, 5):
+        b, s, h, lens = mw2.config_shape(cfg)
+        shape = mla.make_shape(b, s, h, int((lens.max() + 63) // 64), 1, causal=(cfg == 5))
+        host = mla.mla_plan_schedule_host(shape, torch.from_numpy(lens), 148)
+        dev = torch.empty(host.numel(), dtype=torch.int32, device="cuda")
+        mla.mla_get_schedule(shape, torch.from_numpy(lens).cuda(), 148, dev)
+        torch.cuda.synchronize()
+        assert torch.equal(dev.cpu(), host)
+
+
+def test_bad_page_id_is_flagged_not_faulted():
+    wl = mw.make(2, 1, 128, [100, 100], seed=12)
+    wl.block_table[1, 1] = 10 ** 6          # beyond the pool: skipped and flagged
+    O, L, st = run(wl)
+    assert st == -6                         # MLA_ERR_DEVICE_CHECK
+    O_ref, L_ref = oracle.decode(mw.make(2, 1, 128, [100, 100], seed=12))
+    assert_parity(compare(O[:1], L[:1], O_ref[:1], L_ref[:1]), "unaffected request")
+
+
+# ---- the five workloads at full size, sampled rows -------------------------
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_full_size_configs_sampled(cfg):
+    check_sampled(mw.make_config(cfg), n=4)
