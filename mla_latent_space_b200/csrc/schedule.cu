@@ -47,6 +47,7 @@ MLA_HD int first_worker_ge(const int32_t* workers, int W, int64_t key) {
 }
 
 MLA_HD void fill_header(int32_t* hdr, const ShapeInfo& s, int W, int num_tiles) {
+  for (int i = 0; i < kHeaderInts; ++i) hdr[i] = 0;
   hdr[H_MAGIC] = kSchedMagic;
   hdr[H_WORKERS] = W;
   hdr[H_TILES] = num_tiles;
@@ -58,12 +59,15 @@ MLA_HD void fill_header(int32_t* hdr, const ShapeInfo& s, int W, int num_tiles) 
   hdr[H_MAX_PAGES] = s.max_pages;
 }
 
-// Worker w's start position; workers past the end start at (num_tiles, 0).
+// Worker w's start position.  Only min(W, total) workers get work, so the
+// start positions floor(total*w/W_eff) are strictly increasing and an
+// interior page boundary is never shared by two workers; the remaining
+// workers start (and end) at (num_tiles, 0).
 MLA_HD void worker_start(const int32_t* tiles, int num_tiles, int64_t total, int w, int W,
                          int* tile, int* page) {
-  int64_t x = total * w / W;
-  if (total == 0 || x >= total) { *tile = num_tiles; *page = 0; return; }
-  map_position(tiles, num_tiles, x, tile, page);
+  const int64_t We = total < W ? total : W;
+  if (w >= We) { *tile = num_tiles; *page = 0; return; }
+  map_position(tiles, num_tiles, total * w / We, tile, page);
 }
 
 constexpr int kSchedThreads = 1024;

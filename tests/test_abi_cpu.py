@@ -200,6 +200,14 @@ def test_schedule_jagged_and_special_lengths():
     check_schedule([0, 0, 0], 1, 128, False, 148)
 
 
+@pytest.mark.parametrize("lens,n_sms", [([63, 64, 65], 148), ([100, 100], 148), ([256, 256], 148),
+                                        ([3000, 64, 1, 2500], 1000), ([1], 4000)])
+def test_schedule_more_workers_than_work(lens, n_sms):
+    # fewer cost units than workers: the idle workers must not count as pieces
+    check_schedule(lens, 1, 128, False, n_sms)
+    check_schedule(lens, 1, 16, False, n_sms)
+
+
 def test_schedule_spec_causal_and_packed_rows():
     check_schedule([4096] * 32, 16, 128, True, 148)
     check_schedule([5, 17, 16, 100], 16, 16, True, 20)   # 2 query tokens per 128-row tile
