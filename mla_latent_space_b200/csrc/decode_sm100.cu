@@ -1,9 +1,581 @@
-// Placeholder launcher: routes to the SIMT kernel until the tcgen05 kernel
-// lands in this file.
-#include "common.cuh"
-#include <cuda_runtime.h>
+// tcgen05 decode kernel for B200 (sm_100a): MLA decode in absorbed latent
+// space ("MLA Cost Analysis & Regime Guide", section "Absorption Trick":
+// S = scale * Qz . C^T over the 576-d cache rows, O = softmax(S) . C[:, :512]).
+//
+// Why a CTA pair.  One tile is 128 (query token, head) rows.  Its fp32
+// output accumulator, 128 x 512, is exactly the 256 KB of tensor memory
+// (TMEM) of one SM, and its query block, 128 x 576 bf16 = 144 KB, does not
+// fit beside two KV pages in shared memory.  So the work of a tile is split
+// by role across the two SMs of a 2-CTA cluster, each doing full-width
+// (M = 128) MMAs and no work twice:
+//
+//   CTA 0 ("score"): Q lives in its TMEM as the A operand (288 columns);
+//     a TMA warp gathers 64-token pages of the paged cache (9 boxes of
+//     64 x 64 bf16, 128-byte swizzle) into a 3-stage ring; one thread issues
+//     S = Q . page^T (M=128, N=64, K=576) into a double-buffered TMEM
+//     accumulator; a warpgroup (thread = row) runs the online softmax in
+//     the log2 domain with a lazy max (the running max moves only when a
+//     page's max exceeds it by 8, so P <= 256 and fits fp16), and writes P
+//     as fp16 plus per-row rescale factors straight into CTA 1's shared
+//     memory (distributed shared memory), then arrives on CTA 1's barrier.
+//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM; converter warps
+//     load the page's 512 value columns from global memory, convert bf16 ->
+//     fp16 (exact in fp16's normal range) and store them in the 128-byte
+//     swizzled N-major layout; one thread issues O += P . V (M=128, N=256,
+//     K=16, twice per 16 tokens); a warpgroup applies the rare rescales to
+//     O between MMAs and writes the normalised result at the end of a piece.
+//
+// P is fp16 rather than bf16 because rounding P to bf16 alone costs about
+// 1e-3 of relative L1 error in O; fp16 keeps it near 2e-4.  The MMA needs
+// both operands of one type, hence the fp16 copy of V.
+//
+// Every wait is bounded: a wait that runs out sets a status bit in the
+// workspace, tells the peer CTA to stop, and the kernel drains its
+// in-flight copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kernel_util.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
+
+namespace {
+
+using namespace ptx;
+
+constexpr int NZ = 3;  // KV page stages in the score CTA
+constexpr int NS = 2;  // S accumulators in TMEM
+constexpr int NP = 2;  // P stages in the output CTA
+constexpr int NV = 2;  // V stages in the output CTA
+constexpr int kThreads = 512;
+constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
+constexpr uint32_t kPageBytes = 9 * kBox;             // 64 tokens x 576 bf16
+constexpr uint32_t kVStage = 8 * kBox;                // 64 tokens x 512 fp16
+constexpr uint32_t kPStage = 128 * 128;               // 128 rows x 64 fp16
+constexpr uint32_t kTmemS = 320;                      // first S accumulator column
+constexpr uint64_t kTimeoutNs = 2000000000ull;        // a wait gives up after 2 s
+constexpr float kLazyMax = 8.0f;                      // log2 units
+
+struct Bars {
+  uint64_t z_full[NZ], z_empty[NZ], s_full[NS], s_empty[NS], q_ready, p_free[NP];
+  uint64_t v_full[NV], v_empty[NV], p_full[NP], corr_done[NP], o_free, mma_done;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct Meta {               // per P stage, in the output CTA
+  float alpha[128];         // O rescale factor per row
+  float lfin[128];          // softmax denominator (last page of a piece)
+  int32_t flag[4];          // any row of the lane quarter needs a rescale
+  int32_t pad[4];
+};
+
+constexpr uint32_t kOffData = 1024;
+constexpr uint32_t kOffZ = kOffData;
+constexpr uint32_t kOffV = kOffData;
+constexpr uint32_t kOffP = kOffV + NV * kVStage;
+constexpr uint32_t kOffMeta = kOffP + NP * kPStage;
+constexpr uint32_t kSmemS = kOffZ + NZ * kPageBytes;
+constexpr uint32_t kSmemO = kOffMeta + NP * sizeof(Meta);
+constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // + alignment slack
+static_assert(sizeof(Bars) <= kOffData, "barrier block");
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+// Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
+//   QK: A = Q bf16 (TMEM), B = cache page bf16 K-major, N = 64
+//   PV: A = P fp16 K-major (smem), B = V fp16 N-major (smem), N = 256
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((256u >> 3) << 17) |
+                              ((128u >> 4) << 24);
+
+// Shared-memory matrix descriptor, 128-byte swizzle.  lbo / sbo in bytes.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((addr >> 4) & 0x3FFF) | (uint64_t((lbo >> 4) & 0x3FFF) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+struct Params {
+  const uint16_t* q;
+  const uint8_t* kv;
+  const int32_t* block_table;
+  const int32_t* seqlens;
+  const void* sched;
+  void* ws;
+  __nv_bfloat16* out;
+  float* lse;
+  float scale_log2;   // softmax_scale * log2(e)
+  int num_pages;
+  int cap_slots;
+};
+
+struct Ctl {
+  volatile int32_t* abort;
+  uint32_t peer_abort;
+  void* ws;
+};
+
+__device__ __noinline__ void trip(const Ctl& c) {
+  *c.abort = 1;
+  st_cluster_u32(c.peer_abort, 1);
+  flag_status(c.ws, kStatusTimeout);
+}
+
+// Bounded wait on an mbarrier phase; false when this CTA is aborting.
+__device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 31) == 0) {
+      if (*c.abort) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        trip(c);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane polls, and the warp gives up
+// together if any lane gave up (so no lane is left at a warp collective).
+__device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  const bool ok = bwait(c, bar, parity);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (used while draining).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kTimeoutNs) return;
+  }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Calls f(piece) for every piece of every worker this cluster owns; stops
+// when f returns false.
+template <class F>
+__device__ __forceinline__ void each_piece(const SchedView& sv, F&& f) {
+  const int ncl = int(nclusters_x());
+  for (int w = int(cluster_id_x()); w < sv.W; w += ncl) {
+    PieceIter it(sv, w);
+    Piece pc;
+    while (it.next(&pc))
+      if (!f(pc)) return;
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  Bars* bars = reinterpret_cast<Bars*>(gbase);
+  auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const SchedView sv(p.sched);
+  const int rows_total = sv.s_q * sv.heads;
+
+  if (tid == 0) {
+    for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
+    for (int s = 0; s < NS; ++s) { mbar_init(bar(bars->s_full[s]), 1); mbar_init(bar(bars->s_empty[s]), 128); }
+    mbar_init(bar(bars->q_ready), 128);
+    for (int s = 0; s < NP; ++s) {
+      mbar_init(bar(bars->p_free[s]), 1);
+      mbar_init(bar(bars->p_full[s]), 128);
+      mbar_init(bar(bars->corr_done[s]), 128);
+    }
+    for (int s = 0; s < NV; ++s) { mbar_init(bar(bars->v_full[s]), 256); mbar_init(bar(bars->v_empty[s]), 1); }
+    mbar_init(bar(bars->o_free), 128);
+    mbar_init(bar(bars->mma_done), 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0 && rank == 0) tma_prefetch_desc(&tmap);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  cluster_sync();
+
+  Ctl ctl{&bars->abort, mapa(smem_u32(&bars->abort), rank ^ 1u), p.ws};
+
+  if (rank == 0) {
+    // ======================= score CTA =======================
+    if (warp == 0) {
+      if (lane == 0) {  // ---- TMA producer
+        uint32_t zc = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          const int r = pc.T / sv.tiles_per_req;
+          for (int j = pc.p0; j < pc.p1; ++j, ++zc) {
+            const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
+            if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+            int page = p.block_table[size_t(r) * sv.max_pages + j];
+            if (page < 0 || page >= p.num_pages) {
+              flag_status(p.ws, kStatusBadPage);
+              page = 0;   // any valid page; the softmax masks every token of it
+            }
+            const uint32_t fb = bar(bars->z_full[s]);
+            mbar_arrive_expect_tx(fb, kPageBytes);
+            const uint32_t dst = sbase + kOffZ + s * kPageBytes;
+#pragma unroll
+            for (int c = 0; c < 9; ++c) tma_load_3d(dst + c * kBox, &tmap, 64 * c, 0, page, fb);
+          }
+          return true;
+        });
+        // copies still in flight must land before the CTA can leave
+        const uint32_t n = zc < NZ ? zc : NZ;
+        for (uint32_t k = 1; k <= n; ++k) {
+          const uint32_t idx = zc - k;
+          drain_wait(bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {  // ---- QK^T issuer
+        uint32_t zc = 0, sc = 0, pieces = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          if (!bwait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
+          ++pieces;
+          tc_fence_after();
+          for (int j = pc.p0; j < pc.p1; ++j, ++zc, ++sc) {
+            const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
+            const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
+            if (!bwait(ctl, bar(bars->z_full[zs]), zph)) return false;
+            if (!bwait(ctl, bar(bars->s_empty[sb]), sph ^ 1u)) return false;
+            tc_fence_after();
+            const uint32_t d = tmem + kTmemS + 64u * sb;
+            const uint32_t za = sbase + kOffZ + zs * kPageBytes;
+#pragma unroll
+            for (int k = 0; k < 36; ++k)
+              mma_ts(d, tmem + 8u * k, sdesc(za + (k >> 2) * kBox + (k & 3) * 32, 16, 1024), kIdescQK, k > 0);
+            mma_commit(bar(bars->z_empty[zs]));
+            mma_commit(bar(bars->s_full[sb]));
+          }
+          return true;
+        });
+        mma_commit(bar(bars->mma_done));
+        drain_wait(bar(bars->mma_done), 0);
+      }
+    } else if (warp >= 4 && warp < 8) {
+      // ---- softmax warpgroup: thread i owns row i of the tile (TMEM lane i)
+      const int i = tid - 128, wq = warp - 4;
+      const uint32_t lane_off = uint32_t(wq * 32) << 16;
+      const uint32_t o_p = mapa(sbase + kOffP, 1);
+      const uint32_t o_meta = mapa(sbase + kOffMeta, 1);
+      const uint32_t o_pfull = mapa(bar(bars->p_full[0]), 1);
+      uint32_t sc = 0, pcnt = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
+        const int rho = qt * MLA_TILE_ROWS + i;
+        const bool valid = rho < rows_total;
+        int t = p.seqlens[r];
+        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
+        const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
+        // query row -> TMEM lane i, columns [0, 288) (bf16 pairs)
+        {
+          const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (size_t(r) * rows_total + (valid ? rho : 0)) * MLA_D_QK);
+#pragma unroll 1
+          for (int c3 = 0; c3 < 3; ++c3) {
+            uint32_t v[3][32];
+#pragma unroll
+            for (int u = 0; u < 24; ++u) {
+              uint4 x = valid ? ld_global_nc_v4(qrow + c3 * 24 + u) : make_uint4(0, 0, 0, 0);
+              v[u / 8][(u % 8) * 4 + 0] = x.x;
+              v[u / 8][(u % 8) * 4 + 1] = x.y;
+              v[u / 8][(u % 8) * 4 + 2] = x.z;
+              v[u / 8][(u % 8) * 4 + 3] = x.w;
+            }
+#pragma unroll
+            for (int c = 0; c < 3; ++c) tmem_st32(tmem + lane_off + 32u * (c3 * 3 + c), v[c]);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(bars->q_ready));
+        }
+        float m = -INFINITY, l = 0.f;
+        for (int j = pc.p0; j < pc.p1; ++j, ++sc, ++pcnt) {
+          const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
+          if (!wwait(ctl, bar(bars->s_full[sb]), sph)) return false;
+          tc_fence_after();
+          uint32_t sv0[32], sv1[32];
+          tmem_ld32(tmem + lane_off + kTmemS + 64u * sb, sv0);
+          tmem_ld32(tmem + lane_off + kTmemS + 64u * sb + 32u, sv1);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(bars->s_empty[sb]));
+
+          const int page = p.block_table[size_t(r) * sv.max_pages + j];
+          const bool page_ok = page >= 0 && page < p.num_pages;
+          const int nv = page_ok ? Lrow - j * MLA_PAGE_SIZE : 0;   // visible tokens of this row here
+          float x[64];
+          float mb = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[c] = c < nv ? __uint_as_float(sv0[c]) * p.scale_log2 : -INFINITY;
+            x[c + 32] = c + 32 < nv ? __uint_as_float(sv1[c]) * p.scale_log2 : -INFINITY;
+            mb = fmaxf(mb, fmaxf(x[c], x[c + 32]));
+          }
+          float m_new = m, alpha = 1.f;
+          bool need = false;
+          if (mb > m + kLazyMax) {
+            m_new = mb;
+            alpha = ex2(m - m_new);            // 0 when m = -inf
+            need = (j != pc.p0) && (m != -INFINITY);
+          }
+          const bool live = m_new != -INFINITY;
+          const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
+          if (!wwait(ctl, bar(bars->p_free[ps]), pph ^ 1u)) return false;
+          const uint32_t prow = o_p + ps * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
+          float psum = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float e[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              e[u] = live ? ex2(x[8 * k + u] - m_new) : 0.f;
+              psum += e[u];
+            }
+            st_cluster_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(e[0], e[1]), pack_f16(e[2], e[3]),
+                          pack_f16(e[4], e[5]), pack_f16(e[6], e[7]));
+          }
+          l = l * alpha + psum;
+          m = m_new;
+          const uint32_t meta = o_meta + ps * uint32_t(sizeof(Meta));
+          st_cluster_u32(meta + offsetof(Meta, alpha) + 4 * i, __float_as_uint(need ? alpha : 1.f));
+          if (j == pc.p1 - 1) st_cluster_u32(meta + offsetof(Meta, lfin) + 4 * i, __float_as_uint(l));
+          const uint32_t any = __any_sync(0xffffffffu, need) ? 1u : 0u;
+          if (lane == 0) st_cluster_u32(meta + offsetof(Meta, flag) + 4 * wq, any);
+          fence_proxy_async_cluster();
+          mbar_arrive_remote(o_pfull + ps * 8);
+        }
+        if (valid) {
+          const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          if (sv.tile_splits(pc.T) == 1) {
+            p.lse[size_t(r) * rows_total + rho] = lse_v;
+          } else {
+            const int slot = sv.tile_slot_base(pc.T) + pc.split;
+            if (slot < p.cap_slots) ws_partial_lse(p.ws, p.cap_slots, slot)[i] = lse_v;
+            else flag_status(p.ws, kStatusWorkspace);
+          }
+        }
+        return true;
+      });
+    }
+  } else {
+    // ======================= output CTA =======================
+    if (warp == 1) {
+      if (lane == 0) {  // ---- PV issuer
+        uint32_t vc = 0, pcnt = 0, pieces = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          if (pieces > 0 && !bwait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
+          ++pieces;
+          for (int j = pc.p0; j < pc.p1; ++j, ++vc, ++pcnt) {
+            const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
+            const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
+            if (!bwait(ctl, bar(bars->v_full[vs]), vph)) return false;
+            if (!bwait(ctl, bar(bars->corr_done[ps]), pph)) return false;
+            if (!bwait(ctl, bar(bars->p_full[ps]), pph)) return false;
+            tc_fence_after();
+            fence_proxy_async_cta();
+            const uint32_t pa = sbase + kOffP + ps * kPStage;
+            const uint32_t va = sbase + kOffV + vs * kVStage;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = sdesc(pa + 32u * k, 16, 1024);
+#pragma unroll
+              for (int n = 0; n < 2; ++n)
+                mma_ss(tmem + 256u * n, ad, sdesc(va + 4u * n * kBox + 2048u * k, kBox, 1024), kIdescPV,
+                       (j > pc.p0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(bars->v_empty[vs]));
+            mma_commit_mc(bar(bars->p_free[ps]), uint16_t(1u));
+          }
+          return true;
+        });
+        mma_commit(bar(bars->mma_done));
+        drain_wait(bar(bars->mma_done), 0);
+      }
+    } else if (warp >= 4 && warp < 8) {
+      // ---- correction / epilogue warpgroup: thread i owns row i of O
+      const int i = tid - 128, wq = warp - 4;
+      const uint32_t lane_off = uint32_t(wq * 32) << 16;
+      uint32_t vc = 0, pcnt = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
+        const int rho = qt * MLA_TILE_ROWS + i;
+        const bool valid = rho < rows_total;
+        float lfin = 0.f;
+        for (int j = pc.p0; j < pc.p1; ++j, ++vc, ++pcnt) {
+          const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
+          if (!wwait(ctl, bar(bars->p_full[ps]), pph)) return false;
+          const volatile Meta* mt = reinterpret_cast<const volatile Meta*>(gbase + kOffMeta + ps * sizeof(Meta));
+          const int flag = mt->flag[wq];
+          const float alpha = mt->alpha[i];
+          if (j == pc.p1 - 1) lfin = mt->lfin[i];
+          if (flag) {
+            // O must hold every earlier page before it is rescaled
+            const uint32_t pv = vc - 1;
+            if (!wwait(ctl, bar(bars->v_empty[pv % NV]), (pv / NV) & 1u)) return false;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 16; ++c) {
+              uint32_t o[32];
+              tmem_ld32(tmem + lane_off + 32u * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+              tmem_st32(tmem + lane_off + 32u * c, o);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          mbar_arrive(bar(bars->corr_done[ps]));
+        }
+        // epilogue: wait for the last PV, normalise, store
+        {
+          const uint32_t pv = vc - 1;
+          if (!wwait(ctl, bar(bars->v_empty[pv % NV]), (pv / NV) & 1u)) return false;
+          tc_fence_after();
+          const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
+          const bool whole = sv.tile_splits(pc.T) == 1;
+          const int slot = whole ? 0 : sv.tile_slot_base(pc.T) + pc.split;
+          const bool slot_ok = whole || slot < p.cap_slots;
+          uint4* dst_b = reinterpret_cast<uint4*>(p.out + (size_t(r) * rows_total + (valid ? rho : 0)) * MLA_D_V);
+          uint4* dst_f = slot_ok && !whole
+                             ? reinterpret_cast<uint4*>(ws_partial_o(p.ws, p.cap_slots, slot) + size_t(i) * MLA_D_V)
+                             : nullptr;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_off + 32u * c, o);
+            tmem_wait_ld();
+            if (valid && slot_ok) {
+              if (whole) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  dst_b[c * 4 + u] = make_uint4(
+                      pack_bf16(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv),
+                      pack_bf16(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv),
+                      pack_bf16(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv),
+                      pack_bf16(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv));
+              } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                  dst_f[c * 8 + u] = make_uint4(__float_as_uint(__uint_as_float(o[4 * u + 0]) * inv),
+                                                __float_as_uint(__uint_as_float(o[4 * u + 1]) * inv),
+                                                __float_as_uint(__uint_as_float(o[4 * u + 2]) * inv),
+                                                __float_as_uint(__uint_as_float(o[4 * u + 3]) * inv));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar(bars->o_free));
+        }
+        return true;
+      });
+    } else if (warp >= 8) {
+      // ---- converters: 256 threads; thread -> one 16-byte column chunk of
+      // 16 tokens of the page
+      const int ct = tid - 256;
+      const int dch = ct & 63, tok0 = ct >> 6;
+      uint32_t vc = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        const int r = pc.T / sv.tiles_per_req;
+        int t = p.seqlens[r];
+        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
+        for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
+          const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
+          if (!wwait(ctl, bar(bars->v_empty[vs]), vph ^ 1u)) return false;
+          const int page = p.block_table[size_t(r) * sv.max_pages + j];
+          const bool ok = page >= 0 && page < p.num_pages;
+          const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
+          const uint8_t* src = p.kv + size_t(ok ? page : 0) * kPageBytes + dch * 16;
+          uint4 buf[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int tok = tok0 + 4 * u;
+            buf[u] = tok < nvalid ? ld_global_nc_v4(src + size_t(tok) * (MLA_D_QK * 2)) : make_uint4(0, 0, 0, 0);
+          }
+          const uint32_t dst = sbase + kOffV + vs * kVStage + (dch >> 3) * kBox;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int tok = tok0 + 4 * u;
+            st_shared_v4(dst + tok * 128 + ((uint32_t(dch & 7) ^ uint32_t(tok & 7)) << 4), bf16x2_to_f16x2(buf[u].x),
+                         bf16x2_to_f16x2(buf[u].y), bf16x2_to_f16x2(buf[u].z), bf16x2_to_f16x2(buf[u].w));
+          }
+          fence_proxy_async_cta();
+          mbar_arrive(bar(bars->v_full[vs]));
+        }
+        return true;
+      });
+    }
+  }
+
+  // ---- teardown: every MMA has completed (mma_done), every TMEM access has
+  // been waited on; free TMEM and leave together with the peer CTA
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  cluster_sync();
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Tensor map over the bf16 page pool viewed as [pages][64 tokens][576]:
+// boxes of 64 columns x 64 tokens x 1 page, 128-byte swizzle.
+bool make_pool_map(CUtensorMap* map, const void* kv, int num_pages) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cuuint64_t(MLA_D_QK), cuuint64_t(MLA_PAGE_SIZE), cuuint64_t(num_pages)};
+  cuuint64_t strides[2] = {cuuint64_t(MLA_D_QK) * 2, cuuint64_t(MLA_D_QK) * 2 * MLA_PAGE_SIZE};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_scale, const int32_t* block_table,
                                const int32_t* seqlens, float scale, const void* sched, void* ws, void* out,
                                float* lse, int num_pages, int fp8, int cap_slots, int grid_ctas,
@@ -15,9 +587,34 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
-  cudaError_t e = launch_decode_simt(q, kv, kv_scale, block_table, seqlens, scale, sched, ws, out, lse,
-                                     shape->num_pages, shape->cache_dtype == MLA_CACHE_FP8_E4M3, cap_slots, sms,
-                                     stream);
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  if (shape->cache_dtype != MLA_CACHE_BF16) {
+    cudaError_t e = launch_decode_simt(q, kv, kv_scale, block_table, seqlens, scale, sched, ws, out, lse,
+                                       shape->num_pages, 1, cap_slots, sms, stream);
+    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  }
+  CUtensorMap map;
+  if (!make_pool_map(&map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  });
+  if (attr_err != cudaSuccess) return MLA_ERR_CUDA;
+  Params prm;
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.kv = static_cast<const uint8_t*>(kv);
+  prm.block_table = block_table;
+  prm.seqlens = seqlens;
+  prm.sched = sched;
+  prm.ws = ws;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.num_pages = shape->num_pages;
+  prm.cap_slots = cap_slots;
+  const int clusters = sms / 2 > 0 ? sms / 2 : 1;
+  decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(map, prm);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
+
 }  // namespace mla
