@@ -3,8 +3,10 @@
 // the row's result is L = ln sum_i e^{lse_i} and O = sum_i e^{lse_i - L} O_i.
 // Tiles that no worker touched (no visible key) get O = 0 and lse = -inf.
 //
-// One warp per row: lanes read the piece lse values, reduce max and sum,
-// then stream the 512 fp32 values of each piece with float4 loads.
+// One warp per row, (tile, 16 row blocks) CTAs of 8 warps: the lanes read
+// the pieces' lse values at once, reduce max and sum with shuffles, then
+// stream the 512 fp32 values of up to four pieces per round with float4
+// loads all in flight together.
 #include "kernel_util.cuh"
 
 namespace mla {
@@ -12,6 +14,7 @@ namespace mla {
 namespace {
 
 constexpr int kWarps = 8;
+constexpr int kRowBlocks = MLA_TILE_ROWS / kWarps;   // 16
 
 __global__ void __launch_bounds__(kWarps * 32)
 combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __nv_bfloat16* __restrict__ out,
@@ -24,59 +27,73 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
   const int r = T / sv.tiles_per_req, qt = T % sv.tiles_per_req;
   const int rows_total = sv.s_q * sv.heads;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int row = blockIdx.y * kWarps + warp;
+  const int rho = qt * MLA_TILE_ROWS + row;
+  if (rho >= rows_total) return;
   const int base = n > 1 ? sv.tile_slot_base(T) : 0;
   if (n > 1 && base + n > cap_slots) {
-    if (threadIdx.x == 0) flag_status(ws, kStatusWorkspace);
+    if (lane == 0) flag_status(ws, kStatusWorkspace);
     return;
   }
-  for (int row = warp; row < MLA_TILE_ROWS; row += kWarps) {
-    const int rho = qt * MLA_TILE_ROWS + row;
-    if (rho >= rows_total) break;
-    __nv_bfloat16* o = out + (size_t(r) * rows_total + rho) * MLA_D_V;
-    if (n == 0) {
-      for (int c = lane; c < MLA_D_V; c += 32) o[c] = __float2bfloat16_rn(0.f);
-      if (lane == 0) lse[size_t(r) * rows_total + rho] = -INFINITY;
-      continue;
-    }
-    float mx = -INFINITY;
-    for (int i = lane; i < n; i += 32) mx = fmaxf(mx, ws_partial_lse(ws, cap_slots, base + i)[row]);
+  __nv_bfloat16* o = out + (size_t(r) * rows_total + rho) * MLA_D_V;
+  if (n == 0) {
+    reinterpret_cast<uint4*>(o)[lane * 2] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(o)[lane * 2 + 1] = make_uint4(0, 0, 0, 0);
+    if (lane == 0) lse[size_t(r) * rows_total + rho] = -INFINITY;
+    return;
+  }
+  float mx = -INFINITY;
+  for (int i = lane; i < n; i += 32) mx = fmaxf(mx, ws_partial_lse(ws, cap_slots, base + i)[row]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float sum = 0.f;
-    if (mx != -INFINITY)
-      for (int i = lane; i < n; i += 32) sum += __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - mx);
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float sum = 0.f;
+  if (mx != -INFINITY)
+    for (int i = lane; i < n; i += 32) sum += __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - mx);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const float L = (mx == -INFINITY || sum <= 0.f) ? -INFINITY : mx + logf(sum);
-    float4 acc[MLA_D_V / 128];
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float L = (mx == -INFINITY || sum <= 0.f) ? -INFINITY : mx + logf(sum);
+  float4 acc[MLA_D_V / 128];
 #pragma unroll
-    for (int c = 0; c < MLA_D_V / 128; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (L != -INFINITY) {
-      for (int i = 0; i < n; ++i) {
-        const float w = __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - L);
-        if (w == 0.f) continue;
-        const float4* src = reinterpret_cast<const float4*>(ws_partial_o(ws, cap_slots, base + i) + size_t(row) * MLA_D_V);
+  for (int c = 0; c < MLA_D_V / 128; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (L != -INFINITY) {
+    for (int i0 = 0; i0 < n; i0 += 4) {
+      float4 v[4][MLA_D_V / 128];
+      float w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k;
+        w[k] = 0.f;
+        if (i < n) {
+          w[k] = __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - L);
+          const float4* src =
+              reinterpret_cast<const float4*>(ws_partial_o(ws, cap_slots, base + i) + size_t(row) * MLA_D_V);
+#pragma unroll
+          for (int c = 0; c < MLA_D_V / 128; ++c) v[k][c] = __ldcs(src + lane + 32 * c);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (w[k] == 0.f) continue;
 #pragma unroll
         for (int c = 0; c < MLA_D_V / 128; ++c) {
-          float4 v = src[lane + 32 * c];
-          acc[c].x = fmaf(w, v.x, acc[c].x);
-          acc[c].y = fmaf(w, v.y, acc[c].y);
-          acc[c].z = fmaf(w, v.z, acc[c].z);
-          acc[c].w = fmaf(w, v.w, acc[c].w);
+          acc[c].x = fmaf(w[k], v[k][c].x, acc[c].x);
+          acc[c].y = fmaf(w[k], v[k][c].y, acc[c].y);
+          acc[c].z = fmaf(w[k], v[k][c].z, acc[c].z);
+          acc[c].w = fmaf(w[k], v[k][c].w, acc[c].w);
         }
       }
     }
-#pragma unroll
-    for (int c = 0; c < MLA_D_V / 128; ++c) {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[c].x, acc[c].y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[c].z, acc[c].w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      reinterpret_cast<uint2*>(o)[lane + 32 * c] = pk;
-    }
-    if (lane == 0) lse[size_t(r) * rows_total + rho] = L;
   }
+#pragma unroll
+  for (int c = 0; c < MLA_D_V / 128; ++c) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[c].x, acc[c].y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[c].z, acc[c].w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(o)[lane + 32 * c] = pk;
+  }
+  if (lane == 0) lse[size_t(r) * rows_total + rho] = L;
 }
 
 }  // namespace
@@ -84,8 +101,8 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
 cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
                            int cap_slots, cudaStream_t stream) {
   if (num_tiles == 0) return cudaSuccess;
-  combine_kernel<<<num_tiles, kWarps * 32, 0, stream>>>(sched, ws, static_cast<__nv_bfloat16*>(out), lse,
-                                                        cap_slots);
+  combine_kernel<<<dim3(num_tiles, kRowBlocks), kWarps * 32, 0, stream>>>(
+      sched, ws, static_cast<__nv_bfloat16*>(out), lse, cap_slots);
   return cudaGetLastError();
 }
 

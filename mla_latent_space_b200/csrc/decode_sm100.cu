@@ -9,21 +9,23 @@
 // by role across the two SMs of a 2-CTA cluster, each doing full-width
 // (M = 128) MMAs and no work twice:
 //
-//   CTA 0 ("score"): Q lives in its TMEM as the A operand (288 columns);
-//     a TMA warp gathers 64-token pages of the paged cache (9 boxes of
-//     64 x 64 bf16, 128-byte swizzle) into a 3-stage ring; one thread issues
-//     S = Q . page^T (M=128, N=64, K=576) into a double-buffered TMEM
-//     accumulator; a warpgroup (thread = row) runs the online softmax in
+//   CTA 0 ("score"): Q lives in its TMEM as the A operand (288 columns).
+//     A TMA warp gathers 64-token pages of the paged cache (9 boxes of
+//     64 x 64 bf16, 128-byte swizzle) into a 3-stage ring.  One thread
+//     issues S = Q . page^T (M=128, N=64, K=576) into a triple-buffered TMEM
+//     accumulator.  A warpgroup (thread = row) runs the online softmax in
 //     the log2 domain with a lazy max (the running max moves only when a
-//     page's max exceeds it by 8, so P <= 256 and fits fp16), and writes P
-//     as fp16 plus per-row rescale factors straight into CTA 1's shared
-//     memory (distributed shared memory), then arrives on CTA 1's barrier.
-//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM; converter warps
-//     load the page's 512 value columns from global memory, convert bf16 ->
-//     fp16 (exact in fp16's normal range) and store them in the 128-byte
-//     swizzled N-major layout; one thread issues O += P . V (M=128, N=256,
-//     K=16, twice per 16 tokens); a warpgroup applies the rare rescales to
-//     O between MMAs and writes the normalised result at the end of a piece.
+//     page's max exceeds it by 8, so P <= 256 and fits fp16) and writes P as
+//     fp16 plus per-row rescale factors into CTA 1's shared memory over
+//     distributed shared memory (DSMEM).  Eight converter warps read the
+//     page's 512 value columns from the same TMA tile, convert bf16 -> fp16
+//     (exact in fp16's normal range) and push them to CTA 1 the same way, in
+//     the same swizzled layout, so no byte of the cache is read twice from
+//     global memory.
+//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  One thread issues
+//     O += P . V (M=128, N=256, K=16, twice per 16 tokens) from the pushed
+//     stages; a warpgroup applies the rare rescales to O between MMAs and
+//     writes the normalised result at the end of a piece.
 //
 // P is fp16 rather than bf16 because rounding P to bf16 alone costs about
 // 1e-3 of relative L1 error in O; fp16 keeps it near 2e-4.  The MMA needs
@@ -47,9 +49,8 @@ namespace {
 using namespace ptx;
 
 constexpr int NZ = 3;  // KV page stages in the score CTA
-constexpr int NS = 2;  // S accumulators in TMEM
-constexpr int NP = 2;  // P stages in the output CTA
-constexpr int NV = 2;  // V stages in the output CTA
+constexpr int NS = 3;  // S accumulators in TMEM
+constexpr int NX = 2;  // V + P stages in the output CTA
 constexpr int kThreads = 512;
 constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
 constexpr uint32_t kPageBytes = 9 * kBox;             // 64 tokens x 576 bf16
@@ -58,31 +59,37 @@ constexpr uint32_t kPStage = 128 * 128;               // 128 rows x 64 fp16
 constexpr uint32_t kTmemS = 320;                      // first S accumulator column
 constexpr uint64_t kTimeoutNs = 2000000000ull;        // a wait gives up after 2 s
 constexpr float kLazyMax = 8.0f;                      // log2 units
+constexpr int kConvThreads = 256;                     // score-CTA warps 8..15
 
 struct Bars {
-  uint64_t z_full[NZ], z_empty[NZ], s_full[NS], s_empty[NS], q_ready, p_free[NP];
-  uint64_t v_full[NV], v_empty[NV], p_full[NP], corr_done[NP], o_free, mma_done;
+  // score CTA
+  uint64_t z_full[NZ], z_empty[NZ], s_full[NS], s_empty[NS], q_ready, x_free[NX];
+  // output CTA
+  uint64_t v_full[NX], p_full[NX], corr_done[NX], pv_done[NX], o_free;
+  // both
+  uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort;
 };
 
-struct Meta {               // per P stage, in the output CTA
+struct Meta {               // per stage, in the output CTA
   float alpha[128];         // O rescale factor per row
   float lfin[128];          // softmax denominator (last page of a piece)
   int32_t flag[4];          // any row of the lane quarter needs a rescale
-  int32_t pad[4];
 };
 
 constexpr uint32_t kOffData = 1024;
 constexpr uint32_t kOffZ = kOffData;
 constexpr uint32_t kOffV = kOffData;
-constexpr uint32_t kOffP = kOffV + NV * kVStage;
-constexpr uint32_t kOffMeta = kOffP + NP * kPStage;
+constexpr uint32_t kOffP = kOffV + NX * kVStage;
+constexpr uint32_t kOffMeta = kOffP + NX * kPStage;
 constexpr uint32_t kSmemS = kOffZ + NZ * kPageBytes;
-constexpr uint32_t kSmemO = kOffMeta + NP * sizeof(Meta);
+constexpr uint32_t kSmemO = kOffMeta + NX * sizeof(Meta);
 constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // + alignment slack
 static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(sizeof(Meta) % 16 == 0, "meta alignment");
+static_assert(kTmemS + 64 * NS <= 512, "TMEM columns");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
 //   QK: A = Q bf16 (TMEM), B = cache page bf16 K-major, N = 64
@@ -169,6 +176,12 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 // Calls f(piece) for every piece of every worker this cluster owns; stops
 // when f returns false.
 template <class F>
@@ -197,15 +210,19 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   const int rows_total = sv.s_q * sv.heads;
 
   if (tid == 0) {
-    for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
+    for (int s = 0; s < NZ; ++s) {
+      mbar_init(bar(bars->z_full[s]), 1);
+      mbar_init(bar(bars->z_empty[s]), 1 + kConvThreads);   // QK commit + converters
+    }
     for (int s = 0; s < NS; ++s) { mbar_init(bar(bars->s_full[s]), 1); mbar_init(bar(bars->s_empty[s]), 128); }
     mbar_init(bar(bars->q_ready), 128);
-    for (int s = 0; s < NP; ++s) {
-      mbar_init(bar(bars->p_free[s]), 1);
+    for (int s = 0; s < NX; ++s) {
+      mbar_init(bar(bars->x_free[s]), 1);
+      mbar_init(bar(bars->v_full[s]), kConvThreads);
       mbar_init(bar(bars->p_full[s]), 128);
       mbar_init(bar(bars->corr_done[s]), 128);
+      mbar_init(bar(bars->pv_done[s]), 1);
     }
-    for (int s = 0; s < NV; ++s) { mbar_init(bar(bars->v_full[s]), 256); mbar_init(bar(bars->v_empty[s]), 1); }
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
@@ -237,7 +254,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
             int page = p.block_table[size_t(r) * sv.max_pages + j];
             if (page < 0 || page >= p.num_pages) {
               flag_status(p.ws, kStatusBadPage);
-              page = 0;   // any valid page; the softmax masks every token of it
+              page = 0;   // any valid page; the consumers mask every token of it
             }
             const uint32_t fb = bar(bars->z_full[s]);
             mbar_arrive_expect_tx(fb, kPageBytes);
@@ -287,7 +304,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
       const uint32_t o_p = mapa(sbase + kOffP, 1);
       const uint32_t o_meta = mapa(sbase + kOffMeta, 1);
       const uint32_t o_pfull = mapa(bar(bars->p_full[0]), 1);
-      uint32_t sc = 0, pcnt = 0;
+      uint32_t sc = 0, xc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
@@ -295,7 +312,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         int t = p.seqlens[r];
         t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
-        // query row -> TMEM lane i, columns [0, 288) (bf16 pairs)
+        // query row -> TMEM lane i, columns [0, 288) (bf16 pairs).  Every
+        // QK MMA of the previous piece has completed: its last S was read.
         {
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (size_t(r) * rows_total + (valid ? rho : 0)) * MLA_D_QK);
 #pragma unroll 1
@@ -317,7 +335,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
           mbar_arrive(bar(bars->q_ready));
         }
         float m = -INFINITY, l = 0.f;
-        for (int j = pc.p0; j < pc.p1; ++j, ++sc, ++pcnt) {
+        for (int j = pc.p0; j < pc.p1; ++j, ++sc, ++xc) {
           const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
           if (!wwait(ctl, bar(bars->s_full[sb]), sph)) return false;
           tc_fence_after();
@@ -347,9 +365,9 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
             need = (j != pc.p0) && (m != -INFINITY);
           }
           const bool live = m_new != -INFINITY;
-          const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
-          if (!wwait(ctl, bar(bars->p_free[ps]), pph ^ 1u)) return false;
-          const uint32_t prow = o_p + ps * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
+          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+          if (!wwait(ctl, bar(bars->x_free[xs]), xph ^ 1u)) return false;
+          const uint32_t prow = o_p + xs * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
           float psum = 0.f;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -364,13 +382,13 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
           }
           l = l * alpha + psum;
           m = m_new;
-          const uint32_t meta = o_meta + ps * uint32_t(sizeof(Meta));
+          const uint32_t meta = o_meta + xs * uint32_t(sizeof(Meta));
           st_cluster_u32(meta + offsetof(Meta, alpha) + 4 * i, __float_as_uint(need ? alpha : 1.f));
           if (j == pc.p1 - 1) st_cluster_u32(meta + offsetof(Meta, lfin) + 4 * i, __float_as_uint(l));
           const uint32_t any = __any_sync(0xffffffffu, need) ? 1u : 0u;
           if (lane == 0) st_cluster_u32(meta + offsetof(Meta, flag) + 4 * wq, any);
           fence_proxy_async_cluster();
-          mbar_arrive_remote(o_pfull + ps * 8);
+          mbar_arrive_remote(o_pfull + xs * 8);
         }
         if (valid) {
           const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -384,25 +402,63 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         }
         return true;
       });
+    } else if (warp >= 8) {
+      // ---- V converters: the first 512 columns of the landed page (boxes
+      // 0..7 of the TMA tile) -> fp16 -> the output CTA's V stage, at the
+      // same byte offsets (same box structure and swizzle).  Rows at or past
+      // the request's length become zero: their bytes may be anything and
+      // 0 * NaN would poison the accumulator.
+      const int ct = tid - 256;
+      const uint32_t o_v = mapa(sbase + kOffV, 1);
+      const uint32_t o_vfull = mapa(bar(bars->v_full[0]), 1);
+      uint32_t zc = 0, xc = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        const int r = pc.T / sv.tiles_per_req;
+        int t = p.seqlens[r];
+        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
+        for (int j = pc.p0; j < pc.p1; ++j, ++zc, ++xc) {
+          const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
+          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+          const int page = p.block_table[size_t(r) * sv.max_pages + j];
+          const bool ok = page >= 0 && page < p.num_pages;
+          const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
+          if (!wwait(ctl, bar(bars->z_full[zs]), zph)) return false;
+          if (!wwait(ctl, bar(bars->x_free[xs]), xph ^ 1u)) return false;
+          const uint32_t src = sbase + kOffZ + zs * kPageBytes;
+          const uint32_t dst = o_v + xs * kVStage;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
+            const int tok = int((off & (kBox - 1)) >> 7);
+            uint4 v = ld_shared_v4(src + off);
+            if (tok >= nvalid) v = make_uint4(0, 0, 0, 0);
+            st_cluster_v4(dst + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                          bf16x2_to_f16x2(v.w));
+          }
+          fence_proxy_async_cluster();
+          mbar_arrive_remote(o_vfull + xs * 8);
+          mbar_arrive(bar(bars->z_empty[zs]));
+        }
+        return true;
+      });
     }
   } else {
     // ======================= output CTA =======================
     if (warp == 1) {
       if (lane == 0) {  // ---- PV issuer
-        uint32_t vc = 0, pcnt = 0, pieces = 0;
+        uint32_t xc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
           if (pieces > 0 && !bwait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
           ++pieces;
-          for (int j = pc.p0; j < pc.p1; ++j, ++vc, ++pcnt) {
-            const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
-            const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
-            if (!bwait(ctl, bar(bars->v_full[vs]), vph)) return false;
-            if (!bwait(ctl, bar(bars->corr_done[ps]), pph)) return false;
-            if (!bwait(ctl, bar(bars->p_full[ps]), pph)) return false;
+          for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
+            const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+            if (!bwait(ctl, bar(bars->v_full[xs]), xph)) return false;
+            if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
+            if (!bwait(ctl, bar(bars->p_full[xs]), xph)) return false;
             tc_fence_after();
             fence_proxy_async_cta();
-            const uint32_t pa = sbase + kOffP + ps * kPStage;
-            const uint32_t va = sbase + kOffV + vs * kVStage;
+            const uint32_t pa = sbase + kOffP + xs * kPStage;
+            const uint32_t va = sbase + kOffV + xs * kVStage;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const uint64_t ad = sdesc(pa + 32u * k, 16, 1024);
@@ -411,8 +467,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
                 mma_ss(tmem + 256u * n, ad, sdesc(va + 4u * n * kBox + 2048u * k, kBox, 1024), kIdescPV,
                        (j > pc.p0 || k > 0) ? 1u : 0u);
             }
-            mma_commit(bar(bars->v_empty[vs]));
-            mma_commit_mc(bar(bars->p_free[ps]), uint16_t(1u));
+            mma_commit(bar(bars->pv_done[xs]));
+            mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
           return true;
         });
@@ -423,23 +479,25 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
       // ---- correction / epilogue warpgroup: thread i owns row i of O
       const int i = tid - 128, wq = warp - 4;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
-      uint32_t vc = 0, pcnt = 0;
+      uint32_t xc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
         const bool valid = rho < rows_total;
         float lfin = 0.f;
-        for (int j = pc.p0; j < pc.p1; ++j, ++vc, ++pcnt) {
-          const uint32_t ps = pcnt % NP, pph = (pcnt / NP) & 1u;
-          if (!wwait(ctl, bar(bars->p_full[ps]), pph)) return false;
-          const volatile Meta* mt = reinterpret_cast<const volatile Meta*>(gbase + kOffMeta + ps * sizeof(Meta));
+        for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
+          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+          if (!wwait(ctl, bar(bars->p_full[xs]), xph)) return false;
+          const volatile Meta* mt = reinterpret_cast<const volatile Meta*>(gbase + kOffMeta + xs * sizeof(Meta));
           const int flag = mt->flag[wq];
           const float alpha = mt->alpha[i];
           if (j == pc.p1 - 1) lfin = mt->lfin[i];
           if (flag) {
-            // O must hold every earlier page before it is rescaled
-            const uint32_t pv = vc - 1;
-            if (!wwait(ctl, bar(bars->v_empty[pv % NV]), (pv / NV) & 1u)) return false;
+            // O must hold every earlier page before it is rescaled.  The
+            // stage's next completion needs this page's corr_done, so the
+            // parity below names PV(page - 1) unambiguously.
+            const uint32_t pv = xc - 1;
+            if (!wwait(ctl, bar(bars->pv_done[pv % NX]), (pv / NX) & 1u)) return false;
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 16; ++c) {
@@ -453,12 +511,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
             tmem_wait_st();
           }
           tc_fence_before();
-          mbar_arrive(bar(bars->corr_done[ps]));
+          mbar_arrive(bar(bars->corr_done[xs]));
         }
         // epilogue: wait for the last PV, normalise, store
         {
-          const uint32_t pv = vc - 1;
-          if (!wwait(ctl, bar(bars->v_empty[pv % NV]), (pv / NV) & 1u)) return false;
+          const uint32_t pv = xc - 1;
+          if (!wwait(ctl, bar(bars->pv_done[pv % NX]), (pv / NX) & 1u)) return false;
           tc_fence_after();
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
           const bool whole = sv.tile_splits(pc.T) == 1;
@@ -494,41 +552,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
           }
           tc_fence_before();
           mbar_arrive(bar(bars->o_free));
-        }
-        return true;
-      });
-    } else if (warp >= 8) {
-      // ---- converters: 256 threads; thread -> one 16-byte column chunk of
-      // 16 tokens of the page
-      const int ct = tid - 256;
-      const int dch = ct & 63, tok0 = ct >> 6;
-      uint32_t vc = 0;
-      each_piece(sv, [&](const Piece& pc) {
-        const int r = pc.T / sv.tiles_per_req;
-        int t = p.seqlens[r];
-        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
-        for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
-          const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
-          if (!wwait(ctl, bar(bars->v_empty[vs]), vph ^ 1u)) return false;
-          const int page = p.block_table[size_t(r) * sv.max_pages + j];
-          const bool ok = page >= 0 && page < p.num_pages;
-          const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
-          const uint8_t* src = p.kv + size_t(ok ? page : 0) * kPageBytes + dch * 16;
-          uint4 buf[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int tok = tok0 + 4 * u;
-            buf[u] = tok < nvalid ? ld_global_nc_v4(src + size_t(tok) * (MLA_D_QK * 2)) : make_uint4(0, 0, 0, 0);
-          }
-          const uint32_t dst = sbase + kOffV + vs * kVStage + (dch >> 3) * kBox;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int tok = tok0 + 4 * u;
-            st_shared_v4(dst + tok * 128 + ((uint32_t(dch & 7) ^ uint32_t(tok & 7)) << 4), bf16x2_to_f16x2(buf[u].x),
-                         bf16x2_to_f16x2(buf[u].y), bf16x2_to_f16x2(buf[u].z), bf16x2_to_f16x2(buf[u].w));
-          }
-          fence_proxy_async_cta();
-          mbar_arrive(bar(bars->v_full[vs]));
         }
         return true;
       });
