@@ -5,27 +5,31 @@
 // Why a CTA pair.  One tile is 128 (query token, head) rows.  Its fp32
 // output accumulator, 128 x 512, is exactly the 256 KB of tensor memory
 // (TMEM) of one SM, and its query block, 128 x 576 bf16 = 144 KB, does not
-// fit beside two KV pages in shared memory.  So the work of a tile is split
-// by role across the two SMs of a 2-CTA cluster, each doing full-width
-// (M = 128) MMAs and no work twice:
+// fit beside a useful KV ring in shared memory.  So the work of a tile is
+// split by role across the two SMs of a 2-CTA cluster, each doing
+// full-width (M = 128) MMAs and no math twice:
 //
-//   CTA 0 ("score"): Q lives in its TMEM as the A operand (288 columns).
-//     A TMA warp gathers 64-token pages of the paged cache (9 boxes of
-//     64 x 64 bf16, 128-byte swizzle) into a 3-stage ring.  One thread
-//     issues S = Q . page^T (M=128, N=64, K=576) into a triple-buffered TMEM
-//     accumulator.  A warpgroup (thread = row) runs the online softmax in
-//     the log2 domain with a lazy max (the running max moves only when a
-//     page's max exceeds it by 8, so P <= 256 and fits fp16) and writes P as
-//     fp16 plus per-row rescale factors into CTA 1's shared memory over
-//     distributed shared memory (DSMEM).  Eight converter warps read the
-//     page's 512 value columns from the same TMA tile, convert bf16 -> fp16
-//     (exact in fp16's normal range) and push them to CTA 1 the same way, in
-//     the same swizzled layout, so no byte of the cache is read twice from
-//     global memory.
-//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  One thread issues
-//     O += P . V (M=128, N=256, K=16, twice per 16 tokens) from the pushed
-//     stages; a warpgroup applies the rare rescales to O between MMAs and
-//     writes the normalised result at the end of a piece.
+//   CTA 0 ("score"): one TMA warp streams, through a 7-deep ring of 24 KB
+//     stages (3 boxes of 64 tokens x 64 columns, 128-byte swizzle), first
+//     the tile's query rows and then the 64-token pages of the paged cache,
+//     and bulk-prefetches the next pages into L2.  The softmax warpgroup
+//     (thread = row) moves the query rows into TMEM, where they stay as the
+//     A operand of S = Q . page^T (M=128, N=64, K=576), issued by one thread
+//     into a triple-buffered TMEM accumulator.  The warpgroup then runs the
+//     online softmax in the log2 domain with a lazy max (the running max
+//     moves only when a page's max exceeds it by 8, so P <= 256 fits fp16),
+//     writes P (fp16, in the output CTA's swizzled layout) and the per-row
+//     rescale factors to a local staging buffer, and one thread ships it to
+//     the output CTA with a single bulk copy over distributed shared memory
+//     that completes on the output CTA's barrier.
+//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  Eight converter
+//     warps read each page's 512 value columns from global memory (L2, where
+//     CTA 0 prefetched them), convert bf16 -> fp16 (exact in fp16's normal
+//     range) and store them in the 128-byte swizzled N-major layout, with
+//     the next page's loads in flight during the store.  One thread issues
+//     O += P . V (M=128, N=256, K=16, twice per 16 tokens); a warpgroup
+//     applies the rare rescales to O between MMAs and writes the normalised
+//     result at the end of a piece.
 //
 // P is fp16 rather than bf16 because rounding P to bf16 alone costs about
 // 1e-3 of relative L1 error in O; fp16 keeps it near 2e-4.  The MMA needs
@@ -48,18 +52,23 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NZ = 3;  // KV page stages in the score CTA
-constexpr int NS = 3;  // S accumulators in TMEM
-constexpr int NX = 2;  // V + P stages in the output CTA
+constexpr int NZ = 7;   // 24 KB stages of the score CTA's ring
+constexpr int NS = 3;   // S accumulators in TMEM
+constexpr int NX = 2;   // V + P stages in the output CTA
+constexpr int kPrefetchPages = 8;                     // L2 prefetch distance
 constexpr int kThreads = 512;
 constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
+constexpr uint32_t kZStage = 3 * kBox;                // 64 rows x 192 columns
 constexpr uint32_t kPageBytes = 9 * kBox;             // 64 tokens x 576 bf16
 constexpr uint32_t kVStage = 8 * kBox;                // 64 tokens x 512 fp16
-constexpr uint32_t kPStage = 128 * 128;               // 128 rows x 64 fp16
+constexpr uint32_t kPBytes = 128 * 128;               // 128 rows x 64 fp16
+constexpr uint32_t kMetaBytes = 1024;                 // alpha[128], lfin[128]
+constexpr uint32_t kPStage = kPBytes + kMetaBytes;    // one bulk copy
 constexpr uint32_t kTmemS = 320;                      // first S accumulator column
 constexpr uint64_t kTimeoutNs = 2000000000ull;        // a wait gives up after 2 s
 constexpr float kLazyMax = 8.0f;                      // log2 units
-constexpr int kConvThreads = 256;                     // score-CTA warps 8..15
+constexpr int kConvThreads = 256;                     // output-CTA warps 8..15
+constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of warps 4..7
 
 struct Bars {
   // score CTA
@@ -72,23 +81,19 @@ struct Bars {
   int32_t abort;
 };
 
-struct Meta {               // per stage, in the output CTA
-  float alpha[128];         // O rescale factor per row
-  float lfin[128];          // softmax denominator (last page of a piece)
-  int32_t flag[4];          // any row of the lane quarter needs a rescale
-};
-
 constexpr uint32_t kOffData = 1024;
+// score CTA
 constexpr uint32_t kOffZ = kOffData;
+constexpr uint32_t kOffStage = kOffZ + NZ * kZStage;          // P staging (local)
+constexpr uint32_t kSmemS = kOffStage + NX * kPStage;
+// output CTA
 constexpr uint32_t kOffV = kOffData;
-constexpr uint32_t kOffP = kOffV + NX * kVStage;
-constexpr uint32_t kOffMeta = kOffP + NX * kPStage;
-constexpr uint32_t kSmemS = kOffZ + NZ * kPageBytes;
-constexpr uint32_t kSmemO = kOffMeta + NX * sizeof(Meta);
+constexpr uint32_t kOffP = kOffV + NX * kVStage;              // P + meta stages
+constexpr uint32_t kSmemO = kOffP + NX * kPStage;
 constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // + alignment slack
 static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(sizeof(Meta) % 16 == 0, "meta alignment");
+static_assert(kPStage % 1024 == 0 && kZStage % 1024 == 0, "swizzle atoms need 1024-byte alignment");
 static_assert(kTmemS + 64 * NS <= 512, "TMEM columns");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
@@ -116,6 +121,7 @@ struct Params {
   float scale_log2;   // softmax_scale * log2(e)
   int num_pages;
   int cap_slots;
+  int q_rows;         // batch * s_q * heads
 };
 
 struct Ctl {
@@ -176,10 +182,11 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
+// Softmax-warpgroup bounded wait: the 128 threads decide together (a thread
+// leaving alone would strand the others at the warpgroup's named barrier).
+__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  const bool ok = bwait(c, bar, parity);
+  return named_bar_and(kSoftmaxBar, 128, ok);
 }
 
 // Calls f(piece) for every piece of every worker this cluster owns; stops
@@ -195,8 +202,13 @@ __device__ __forceinline__ void each_piece(const SchedView& sv, F&& f) {
   }
 }
 
+__device__ __forceinline__ int clamp_len(int t, const SchedView& sv) {
+  return max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_constant__ CUtensorMap q_map,
+                    const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -210,16 +222,13 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   const int rows_total = sv.s_q * sv.heads;
 
   if (tid == 0) {
-    for (int s = 0; s < NZ; ++s) {
-      mbar_init(bar(bars->z_full[s]), 1);
-      mbar_init(bar(bars->z_empty[s]), 1 + kConvThreads);   // QK commit + converters
-    }
+    for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
     for (int s = 0; s < NS; ++s) { mbar_init(bar(bars->s_full[s]), 1); mbar_init(bar(bars->s_empty[s]), 128); }
     mbar_init(bar(bars->q_ready), 128);
     for (int s = 0; s < NX; ++s) {
       mbar_init(bar(bars->x_free[s]), 1);
       mbar_init(bar(bars->v_full[s]), kConvThreads);
-      mbar_init(bar(bars->p_full[s]), 128);
+      mbar_init(bar(bars->p_full[s]), 1);
       mbar_init(bar(bars->corr_done[s]), 128);
       mbar_init(bar(bars->pv_done[s]), 1);
     }
@@ -228,7 +237,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0 && rank == 0) tma_prefetch_desc(&tmap);
+  if (warp == 0 && lane == 0 && rank == 0) {
+    tma_prefetch_desc(&pool_map);
+    tma_prefetch_desc(&q_map);
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
     tmem_relinquish();
@@ -244,23 +256,53 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
   if (rank == 0) {
     // ======================= score CTA =======================
     if (warp == 0) {
-      if (lane == 0) {  // ---- TMA producer
+      if (lane == 0) {  // ---- TMA producer: per piece 6 query stages, then 3 stages per page
         uint32_t zc = 0;
+        auto page_of = [&](int r, int j) {
+          int page = p.block_table[size_t(r) * sv.max_pages + j];
+          return (page < 0 || page >= p.num_pages) ? -1 : page;
+        };
         each_piece(sv, [&](const Piece& pc) {
-          const int r = pc.T / sv.tiles_per_req;
-          for (int j = pc.p0; j < pc.p1; ++j, ++zc) {
-            const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
-            if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
-            int page = p.block_table[size_t(r) * sv.max_pages + j];
-            if (page < 0 || page >= p.num_pages) {
+          const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
+          const int row0 = r * rows_total + qt * MLA_TILE_ROWS;
+          {
+            const int nrows = min(MLA_TILE_ROWS, p.q_rows - row0);
+            prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK, uint32_t(nrows) * MLA_D_QK * 2);
+          }
+          for (int j = pc.p0; j < min(pc.p1, pc.p0 + kPrefetchPages); ++j) {
+            const int pg = page_of(r, j);
+            if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
+          }
+          for (int h = 0; h < 2; ++h) {
+            for (int kc = 0; kc < 3; ++kc, ++zc) {
+              const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
+              if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+              const uint32_t fb = bar(bars->z_full[s]);
+              mbar_arrive_expect_tx(fb, kZStage);
+              const uint32_t dst = sbase + kOffZ + s * kZStage;
+#pragma unroll
+              for (int b = 0; b < 3; ++b) tma_load_2d(dst + b * kBox, &q_map, 192 * kc + 64 * b, row0 + 64 * h, fb);
+            }
+          }
+          for (int j = pc.p0; j < pc.p1; ++j) {
+            if (j + kPrefetchPages < pc.p1) {
+              const int pg = page_of(r, j + kPrefetchPages);
+              if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
+            }
+            int page = page_of(r, j);
+            if (page < 0) {
               flag_status(p.ws, kStatusBadPage);
               page = 0;   // any valid page; the consumers mask every token of it
             }
-            const uint32_t fb = bar(bars->z_full[s]);
-            mbar_arrive_expect_tx(fb, kPageBytes);
-            const uint32_t dst = sbase + kOffZ + s * kPageBytes;
+            for (int kc = 0; kc < 3; ++kc, ++zc) {
+              const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
+              if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+              const uint32_t fb = bar(bars->z_full[s]);
+              mbar_arrive_expect_tx(fb, kZStage);
+              const uint32_t dst = sbase + kOffZ + s * kZStage;
 #pragma unroll
-            for (int c = 0; c < 9; ++c) tma_load_3d(dst + c * kBox, &tmap, 64 * c, 0, page, fb);
+              for (int b = 0; b < 3; ++b) tma_load_3d(dst + b * kBox, &pool_map, 192 * kc + 64 * b, 0, page, fb);
+            }
           }
           return true;
         });
@@ -277,19 +319,25 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         each_piece(sv, [&](const Piece& pc) {
           if (!bwait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
           ++pieces;
+          // the query rows are in TMEM: release their six stages
+          for (int u = 0; u < 6; ++u, ++zc) mbar_arrive(bar(bars->z_empty[zc % NZ]));
           tc_fence_after();
-          for (int j = pc.p0; j < pc.p1; ++j, ++zc, ++sc) {
-            const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
+          for (int j = pc.p0; j < pc.p1; ++j, ++sc) {
             const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
-            if (!bwait(ctl, bar(bars->z_full[zs]), zph)) return false;
             if (!bwait(ctl, bar(bars->s_empty[sb]), sph ^ 1u)) return false;
-            tc_fence_after();
             const uint32_t d = tmem + kTmemS + 64u * sb;
-            const uint32_t za = sbase + kOffZ + zs * kPageBytes;
+            for (int kc = 0; kc < 3; ++kc, ++zc) {
+              const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
+              if (!bwait(ctl, bar(bars->z_full[zs]), zph)) return false;
+              tc_fence_after();
+              const uint32_t za = sbase + kOffZ + zs * kZStage;
 #pragma unroll
-            for (int k = 0; k < 36; ++k)
-              mma_ts(d, tmem + 8u * k, sdesc(za + (k >> 2) * kBox + (k & 3) * 32, 16, 1024), kIdescQK, k > 0);
-            mma_commit(bar(bars->z_empty[zs]));
+              for (int k = 0; k < 12; ++k) {
+                const int kk = 12 * kc + k;
+                mma_ts(d, tmem + 8u * kk, sdesc(za + (k >> 2) * kBox + (k & 3) * 32, 16, 1024), kIdescQK, kk > 0);
+              }
+              mma_commit(bar(bars->z_empty[zs]));
+            }
             mma_commit(bar(bars->s_full[sb]));
           }
           return true;
@@ -302,34 +350,41 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
       const int i = tid - 128, wq = warp - 4;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
       const uint32_t o_p = mapa(sbase + kOffP, 1);
-      const uint32_t o_meta = mapa(sbase + kOffMeta, 1);
       const uint32_t o_pfull = mapa(bar(bars->p_full[0]), 1);
-      uint32_t sc = 0, xc = 0;
+      const uint32_t stg = sbase + kOffStage;
+      uint32_t zc = 0, sc = 0, xc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
         const bool valid = rho < rows_total;
-        int t = p.seqlens[r];
-        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
+        const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
-        // query row -> TMEM lane i, columns [0, 288) (bf16 pairs).  Every
-        // QK MMA of the previous piece has completed: its last S was read.
+        // query row i -> TMEM lane i, columns [0, 288) (bf16 pairs).  Rows
+        // 0-63 are in the piece's first three stages, 64-127 in the next
+        // three; every QK MMA of the previous piece has completed because
+        // its last S was read.
         {
-          const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (size_t(r) * rows_total + (valid ? rho : 0)) * MLA_D_QK);
+          const int h = i >> 6, ri = i & 63;
 #pragma unroll 1
-          for (int c3 = 0; c3 < 3; ++c3) {
-            uint32_t v[3][32];
+          for (int kc = 0; kc < 3; ++kc) {
+            const uint32_t idx = zc + 3 * h + kc;
+            if (!gwait(ctl, bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u)) return false;
+            const uint32_t st = sbase + kOffZ + (idx % NZ) * kZStage + ri * 128;
 #pragma unroll
-            for (int u = 0; u < 24; ++u) {
-              uint4 x = valid ? ld_global_nc_v4(qrow + c3 * 24 + u) : make_uint4(0, 0, 0, 0);
-              v[u / 8][(u % 8) * 4 + 0] = x.x;
-              v[u / 8][(u % 8) * 4 + 1] = x.y;
-              v[u / 8][(u % 8) * 4 + 2] = x.z;
-              v[u / 8][(u % 8) * 4 + 3] = x.w;
+            for (int b = 0; b < 3; ++b) {
+              uint32_t v[32];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const uint4 x = ld_shared_v4(st + b * kBox + ((uint32_t(k) ^ uint32_t(ri & 7)) << 4));
+                v[4 * k + 0] = x.x;
+                v[4 * k + 1] = x.y;
+                v[4 * k + 2] = x.z;
+                v[4 * k + 3] = x.w;
+              }
+              tmem_st32(tmem + lane_off + 32u * (3 * kc + b), v);
             }
-#pragma unroll
-            for (int c = 0; c < 3; ++c) tmem_st32(tmem + lane_off + 32u * (c3 * 3 + c), v[c]);
           }
+          zc += 6 + 3 * (pc.p1 - pc.p0);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
@@ -337,7 +392,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         float m = -INFINITY, l = 0.f;
         for (int j = pc.p0; j < pc.p1; ++j, ++sc, ++xc) {
           const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
-          if (!wwait(ctl, bar(bars->s_full[sb]), sph)) return false;
+          if (!gwait(ctl, bar(bars->s_full[sb]), sph)) return false;
           tc_fence_after();
           uint32_t sv0[32], sv1[32];
           tmem_ld32(tmem + lane_off + kTmemS + 64u * sb, sv0);
@@ -366,8 +421,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
           }
           const bool live = m_new != -INFINITY;
           const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
-          if (!wwait(ctl, bar(bars->x_free[xs]), xph ^ 1u)) return false;
-          const uint32_t prow = o_p + xs * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
+          // staging buffer xs is free once the copy of page xc-2 has read it
+          if (i == 0) bulk_wait_group_read<1>();
+          named_bar_sync(kSoftmaxBar, 128);
+          const uint32_t prow = stg + xs * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
           float psum = 0.f;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -377,18 +434,24 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
               e[u] = live ? ex2(x[8 * k + u] - m_new) : 0.f;
               psum += e[u];
             }
-            st_cluster_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(e[0], e[1]), pack_f16(e[2], e[3]),
-                          pack_f16(e[4], e[5]), pack_f16(e[6], e[7]));
+            st_shared_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(e[0], e[1]), pack_f16(e[2], e[3]),
+                         pack_f16(e[4], e[5]), pack_f16(e[6], e[7]));
           }
           l = l * alpha + psum;
           m = m_new;
-          const uint32_t meta = o_meta + xs * uint32_t(sizeof(Meta));
-          st_cluster_u32(meta + offsetof(Meta, alpha) + 4 * i, __float_as_uint(need ? alpha : 1.f));
-          if (j == pc.p1 - 1) st_cluster_u32(meta + offsetof(Meta, lfin) + 4 * i, __float_as_uint(l));
-          const uint32_t any = __any_sync(0xffffffffu, need) ? 1u : 0u;
-          if (lane == 0) st_cluster_u32(meta + offsetof(Meta, flag) + 4 * wq, any);
-          fence_proxy_async_cluster();
-          mbar_arrive_remote(o_pfull + xs * 8);
+          const uint32_t meta = stg + xs * kPStage + kPBytes;
+          st_shared_u32(meta + 4 * i, __float_as_uint(need ? alpha : 1.f));
+          st_shared_u32(meta + 512 + 4 * i, __float_as_uint(l));
+          fence_proxy_async_cta();
+          // the output CTA's stage xs is free once PV(xc-2) completed; the
+          // barrier also publishes the staging writes to thread 0
+          const bool free_ok = i == 0 ? bwait(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
+          if (!named_bar_and(kSoftmaxBar, 128, free_ok)) return false;
+          if (i == 0) {
+            mbar_arrive_expect_tx_remote(o_pfull + xs * 8, kPStage);
+            bulk_copy_to_peer(o_p + xs * kPStage, stg + xs * kPStage, kPStage, o_pfull + xs * 8);
+            bulk_commit_group();
+          }
         }
         if (valid) {
           const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -402,45 +465,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         }
         return true;
       });
-    } else if (warp >= 8) {
-      // ---- V converters: the first 512 columns of the landed page (boxes
-      // 0..7 of the TMA tile) -> fp16 -> the output CTA's V stage, at the
-      // same byte offsets (same box structure and swizzle).  Rows at or past
-      // the request's length become zero: their bytes may be anything and
-      // 0 * NaN would poison the accumulator.
-      const int ct = tid - 256;
-      const uint32_t o_v = mapa(sbase + kOffV, 1);
-      const uint32_t o_vfull = mapa(bar(bars->v_full[0]), 1);
-      uint32_t zc = 0, xc = 0;
-      each_piece(sv, [&](const Piece& pc) {
-        const int r = pc.T / sv.tiles_per_req;
-        int t = p.seqlens[r];
-        t = max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
-        for (int j = pc.p0; j < pc.p1; ++j, ++zc, ++xc) {
-          const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
-          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
-          const int page = p.block_table[size_t(r) * sv.max_pages + j];
-          const bool ok = page >= 0 && page < p.num_pages;
-          const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
-          if (!wwait(ctl, bar(bars->z_full[zs]), zph)) return false;
-          if (!wwait(ctl, bar(bars->x_free[xs]), xph ^ 1u)) return false;
-          const uint32_t src = sbase + kOffZ + zs * kPageBytes;
-          const uint32_t dst = o_v + xs * kVStage;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
-            const int tok = int((off & (kBox - 1)) >> 7);
-            uint4 v = ld_shared_v4(src + off);
-            if (tok >= nvalid) v = make_uint4(0, 0, 0, 0);
-            st_cluster_v4(dst + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                          bf16x2_to_f16x2(v.w));
-          }
-          fence_proxy_async_cluster();
-          mbar_arrive_remote(o_vfull + xs * 8);
-          mbar_arrive(bar(bars->z_empty[zs]));
-        }
-        return true;
-      });
+      // no copy may still be in flight when the CTAs leave
+      if (i == 0) bulk_wait_group_all();
     }
   } else {
     // ======================= output CTA =======================
@@ -456,7 +482,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
             if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
             if (!bwait(ctl, bar(bars->p_full[xs]), xph)) return false;
             tc_fence_after();
-            fence_proxy_async_cta();
             const uint32_t pa = sbase + kOffP + xs * kPStage;
             const uint32_t va = sbase + kOffV + xs * kVStage;
 #pragma unroll
@@ -488,11 +513,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
           const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
           if (!wwait(ctl, bar(bars->p_full[xs]), xph)) return false;
-          const volatile Meta* mt = reinterpret_cast<const volatile Meta*>(gbase + kOffMeta + xs * sizeof(Meta));
-          const int flag = mt->flag[wq];
-          const float alpha = mt->alpha[i];
-          if (j == pc.p1 - 1) lfin = mt->lfin[i];
-          if (flag) {
+          const volatile float* meta = reinterpret_cast<const volatile float*>(gbase + kOffP + xs * kPStage + kPBytes);
+          const float alpha = meta[i];
+          if (j == pc.p1 - 1) lfin = meta[128 + i];
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
             // O must hold every earlier page before it is rescaled.  The
             // stage's next completion needs this page's corr_done, so the
             // parity below names PV(page - 1) unambiguously.
@@ -555,6 +579,47 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
         }
         return true;
       });
+    } else if (warp >= 8) {
+      // ---- V converters: thread -> one 16-byte column chunk (8 values) of
+      // 16 of the page's 64 tokens.  Global bf16 -> fp16 -> the swizzled
+      // N-major stage.  Tokens at or past the request's length are zero
+      // (their bytes may be anything; 0 * NaN would poison O).  The next
+      // page's loads are issued right after this page's stores.
+      const int ct = tid - 256;
+      const int dch = ct & 63, tok0 = ct >> 6;
+      uint32_t xc = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        const int r = pc.T / sv.tiles_per_req;
+        const int t = clamp_len(p.seqlens[r], sv);
+        uint4 buf[16];
+        auto load = [&](int j) {
+          const int page = p.block_table[size_t(r) * sv.max_pages + j];
+          const bool ok = page >= 0 && page < p.num_pages;
+          const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
+          const uint8_t* src = p.kv + size_t(ok ? page : 0) * kPageBytes + dch * 16;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int tok = tok0 + 4 * u;
+            buf[u] = tok < nvalid ? ld_global_nc_v4(src + size_t(tok) * (MLA_D_QK * 2)) : make_uint4(0, 0, 0, 0);
+          }
+        };
+        load(pc.p0);
+        for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
+          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+          if (!wwait(ctl, bar(bars->pv_done[xs]), xph ^ 1u)) return false;
+          const uint32_t dst = sbase + kOffV + xs * kVStage + (dch >> 3) * kBox;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int tok = tok0 + 4 * u;
+            st_shared_v4(dst + tok * 128 + ((uint32_t(dch & 7) ^ uint32_t(tok & 7)) << 4), bf16x2_to_f16x2(buf[u].x),
+                         bf16x2_to_f16x2(buf[u].y), bf16x2_to_f16x2(buf[u].z), bf16x2_to_f16x2(buf[u].w));
+          }
+          fence_proxy_async_cta();
+          mbar_arrive(bar(bars->v_full[xs]));
+          if (j + 1 < pc.p1) load(j + 1);
+        }
+        return true;
+      });
     }
   }
 
@@ -597,6 +662,21 @@ bool make_pool_map(CUtensorMap* map, const void* kv, int num_pages) {
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over the query rows [batch * s_q * heads][576] bf16: boxes of
+// 64 columns x 64 rows, 128-byte swizzle.  Rows past the end read as zero.
+bool make_q_map(CUtensorMap* map, const void* q, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(MLA_D_QK), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(MLA_D_QK) * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_scale, const int32_t* block_table,
@@ -615,8 +695,9 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
                                        shape->num_pages, 1, cap_slots, sms, stream);
     return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
   }
-  CUtensorMap map;
-  if (!make_pool_map(&map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+  const int q_rows = shape->batch * shape->s_q * shape->num_heads;
+  CUtensorMap pool_map, q_map;
+  if (!make_pool_map(&pool_map, kv, shape->num_pages) || !make_q_map(&q_map, q, q_rows)) return MLA_ERR_CUDA;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
@@ -635,8 +716,9 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.num_pages = shape->num_pages;
   prm.cap_slots = cap_slots;
+  prm.q_rows = q_rows;
   const int clusters = sms / 2 > 0 ? sms / 2 : 1;
-  decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(map, prm);
+  decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(pool_map, q_map, prm);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
