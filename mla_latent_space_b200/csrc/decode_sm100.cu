@@ -9,27 +9,28 @@
 // split by role across the two SMs of a 2-CTA cluster, each doing
 // full-width (M = 128) MMAs and no math twice:
 //
-//   CTA 0 ("score"): one TMA warp streams, through a 7-deep ring of 24 KB
-//     stages (3 boxes of 64 tokens x 64 columns, 128-byte swizzle), first
-//     the tile's query rows and then the 64-token pages of the paged cache,
-//     and bulk-prefetches the next pages into L2.  The softmax warpgroup
-//     (thread = row) moves the query rows into TMEM, where they stay as the
-//     A operand of S = Q . page^T (M=128, N=64, K=576), issued by one thread
-//     into a triple-buffered TMEM accumulator.  The warpgroup then runs the
-//     online softmax in the log2 domain with a lazy max (the running max
-//     moves only when a page's max exceeds it by 8, so P <= 256 fits fp16),
-//     writes P (fp16, in the output CTA's swizzled layout) and the per-row
-//     rescale factors to a local staging buffer, and one thread ships it to
-//     the output CTA with a single bulk copy over distributed shared memory
-//     that completes on the output CTA's barrier.
+//   CTA 0 ("score"): the query rows live in its TMEM (288 columns) as the A
+//     operand of S = Q . C^T.  Keys are taken two pages (128 tokens) at a
+//     time, because an N=64 MMA runs at about half the tensor core's rate
+//     and N=128 at full rate.  One TMA warp streams the query rows and then
+//     each 2-page block through an 11-deep ring of 16 KB stages (one 64-column
+//     box of both pages, 128-byte swizzle) and bulk-prefetches later pages
+//     into L2.  One thread issues 36 MMAs of M=128, N=128, K=16 per block
+//     into a 128-column TMEM accumulator.  Two warpgroups run the online
+//     softmax, one page each (thread = row), exchanging the row max and sum
+//     through shared memory; the running max is lazy (it moves only when a
+//     block's max exceeds it by 8 in log2 units, so P <= 256 fits fp16).
+//     They write P (fp16, in the output CTA's swizzled layout) and per-row
+//     rescale factors to a staging buffer, which one thread ships to the
+//     output CTA with a single bulk copy over distributed shared memory.
 //   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  Eight converter
 //     warps read each page's 512 value columns from global memory (L2, where
 //     CTA 0 prefetched them), convert bf16 -> fp16 (exact in fp16's normal
-//     range) and store them in the 128-byte swizzled N-major layout, with
-//     the next page's loads in flight during the store.  One thread issues
-//     O += P . V (M=128, N=256, K=16, twice per 16 tokens); a warpgroup
-//     applies the rare rescales to O between MMAs and writes the normalised
-//     result at the end of a piece.
+//     range) and store them in the 128-byte swizzled N-major layout, the next
+//     page's loads in flight during the store.  One thread issues
+//     O += P . V (M=128, N=256, K=16, twice per 16 tokens) page by page; a
+//     warpgroup applies the rare rescales to O between blocks and writes the
+//     normalised result at the end of a piece.
 //
 // P is fp16 rather than bf16 because rounding P to bf16 alone costs about
 // 1e-3 of relative L1 error in O; fp16 keeps it near 2e-4.  The MMA needs
@@ -52,29 +53,30 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NZ = 7;   // 24 KB stages of the score CTA's ring
-constexpr int NS = 3;   // S accumulators in TMEM
-constexpr int NX = 2;   // V + P stages in the output CTA
+constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring
+constexpr int NX = 2;   // P block stages (output CTA)
+constexpr int NV = 2;   // V page stages (output CTA)
 constexpr int kPrefetchPages = 8;                     // L2 prefetch distance
 constexpr int kThreads = 512;
 constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
-constexpr uint32_t kZStage = 3 * kBox;                // 64 rows x 192 columns
+constexpr uint32_t kZStage = 2 * kBox;                // one 64-column box of both pages (128 rows)
 constexpr uint32_t kPageBytes = 9 * kBox;             // 64 tokens x 576 bf16
 constexpr uint32_t kVStage = 8 * kBox;                // 64 tokens x 512 fp16
-constexpr uint32_t kPBytes = 128 * 128;               // 128 rows x 64 fp16
-constexpr uint32_t kMetaBytes = 1024;                 // alpha[128], lfin[128]
-constexpr uint32_t kPStage = kPBytes + kMetaBytes;    // one bulk copy
-constexpr uint32_t kTmemS = 320;                      // first S accumulator column
+constexpr uint32_t kPBytes = 2 * 128 * 128;           // 128 rows x 128 fp16 (two pages)
+constexpr uint32_t kMetaBytes = 1024;                 // alpha[128], l[128]
+constexpr uint32_t kPStage = kPBytes + kMetaBytes;    // one bulk copy per block
+constexpr uint32_t kTmemS = 384;                      // S accumulator: columns 384..511
 constexpr uint64_t kTimeoutNs = 2000000000ull;        // a wait gives up after 2 s
 constexpr float kLazyMax = 8.0f;                      // log2 units
 constexpr int kConvThreads = 256;                     // output-CTA warps 8..15
-constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of warps 4..7
+constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
+constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of the softmax warps
 
 struct Bars {
   // score CTA
-  uint64_t z_full[NZ], z_empty[NZ], s_full[NS], s_empty[NS], q_ready, x_free[NX];
+  uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
   // output CTA
-  uint64_t v_full[NX], p_full[NX], corr_done[NX], pv_done[NX], o_free;
+  uint64_t v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], o_free;
   // both
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -84,22 +86,22 @@ struct Bars {
 constexpr uint32_t kOffData = 1024;
 // score CTA
 constexpr uint32_t kOffZ = kOffData;
-constexpr uint32_t kOffStage = kOffZ + NZ * kZStage;          // P staging (local)
-constexpr uint32_t kSmemS = kOffStage + NX * kPStage;
+constexpr uint32_t kOffStage = kOffZ + NZ * kZStage;          // P staging (local, one block)
+constexpr uint32_t kOffXchg = kOffStage + kPStage;            // row max / sum exchange
+constexpr uint32_t kSmemS = kOffXchg + 4 * 128 * 4;
 // output CTA
 constexpr uint32_t kOffV = kOffData;
-constexpr uint32_t kOffP = kOffV + NX * kVStage;              // P + meta stages
+constexpr uint32_t kOffP = kOffV + NV * kVStage;              // P + meta block stages
 constexpr uint32_t kSmemO = kOffP + NX * kPStage;
 constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // + alignment slack
 static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kPStage % 1024 == 0 && kZStage % 1024 == 0, "swizzle atoms need 1024-byte alignment");
-static_assert(kTmemS + 64 * NS <= 512, "TMEM columns");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
-//   QK: A = Q bf16 (TMEM), B = cache page bf16 K-major, N = 64
+//   QK: A = Q bf16 (TMEM), B = cache rows bf16 K-major, N = 128
 //   PV: A = P fp16 K-major (smem), B = V fp16 N-major (smem), N = 256
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((256u >> 3) << 17) |
                               ((128u >> 4) << 24);
 
@@ -159,6 +161,13 @@ __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parit
   return __all_sync(0xffffffffu, ok);
 }
 
+// Softmax-group bounded wait: the 256 threads decide together (a thread
+// leaving alone would strand the others at the group's named barrier).
+__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  const bool ok = bwait(c, bar, parity);
+  return named_bar_and(kSoftmaxBar, kSmThreads, ok);
+}
+
 // Bounded wait that ignores the abort flag (used while draining).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
@@ -182,11 +191,10 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Softmax-warpgroup bounded wait: the 128 threads decide together (a thread
-// leaving alone would strand the others at the warpgroup's named barrier).
-__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  const bool ok = bwait(c, bar, parity);
-  return named_bar_and(kSoftmaxBar, 128, ok);
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // Calls f(piece) for every piece of every worker this cluster owns; stops
@@ -223,19 +231,22 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 
   if (tid == 0) {
     for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
-    for (int s = 0; s < NS; ++s) { mbar_init(bar(bars->s_full[s]), 1); mbar_init(bar(bars->s_empty[s]), 128); }
-    mbar_init(bar(bars->q_ready), 128);
+    mbar_init(bar(bars->s_full), 1);
+    mbar_init(bar(bars->s_empty), kSmThreads);
+    mbar_init(bar(bars->q_ready), kSmThreads);
     for (int s = 0; s < NX; ++s) {
       mbar_init(bar(bars->x_free[s]), 1);
-      mbar_init(bar(bars->v_full[s]), kConvThreads);
       mbar_init(bar(bars->p_full[s]), 1);
       mbar_init(bar(bars->corr_done[s]), 128);
-      mbar_init(bar(bars->pv_done[s]), 1);
     }
+    for (int s = 0; s < NV; ++s) { mbar_init(bar(bars->v_full[s]), kConvThreads); mbar_init(bar(bars->pv_done[s]), 1); }
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
     fence_mbar_init();
+    // the output CTA arms its P stages for their first bulk copy
+    if (rank == 1)
+      for (int s = 0; s < NX; ++s) mbar_arrive_expect_tx(bar(bars->p_full[s]), kPStage);
   }
   if (warp == 0 && lane == 0 && rank == 0) {
     tma_prefetch_desc(&pool_map);
@@ -256,52 +267,52 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   if (rank == 0) {
     // ======================= score CTA =======================
     if (warp == 0) {
-      if (lane == 0) {  // ---- TMA producer: per piece 6 query stages, then 3 stages per page
+      if (lane == 0) {  // ---- TMA producer: 9 query stages per piece, then 9 per 2-page block
         uint32_t zc = 0;
         auto page_of = [&](int r, int j) {
           int page = p.block_table[size_t(r) * sv.max_pages + j];
           return (page < 0 || page >= p.num_pages) ? -1 : page;
         };
+        auto stage = [&](uint32_t tx, uint32_t* dst) -> bool {
+          const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
+          if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+          mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
+          *dst = sbase + kOffZ + s * kZStage;
+          return true;
+        };
         each_piece(sv, [&](const Piece& pc) {
           const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
           const int row0 = r * rows_total + qt * MLA_TILE_ROWS;
-          {
-            const int nrows = min(MLA_TILE_ROWS, p.q_rows - row0);
-            prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK, uint32_t(nrows) * MLA_D_QK * 2);
-          }
+          prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK,
+                           uint32_t(min(MLA_TILE_ROWS, p.q_rows - row0)) * MLA_D_QK * 2);
           for (int j = pc.p0; j < min(pc.p1, pc.p0 + kPrefetchPages); ++j) {
             const int pg = page_of(r, j);
             if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
           }
-          for (int h = 0; h < 2; ++h) {
-            for (int kc = 0; kc < 3; ++kc, ++zc) {
-              const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
-              if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
-              const uint32_t fb = bar(bars->z_full[s]);
-              mbar_arrive_expect_tx(fb, kZStage);
-              const uint32_t dst = sbase + kOffZ + s * kZStage;
-#pragma unroll
-              for (int b = 0; b < 3; ++b) tma_load_2d(dst + b * kBox, &q_map, 192 * kc + 64 * b, row0 + 64 * h, fb);
-            }
+          for (int c = 0; c < 9; ++c, ++zc) {
+            uint32_t dst;
+            if (!stage(kZStage, &dst)) return false;
+            const uint32_t fb = bar(bars->z_full[zc % NZ]);
+            tma_load_2d(dst, &q_map, 64 * c, row0, fb);
+            tma_load_2d(dst + kBox, &q_map, 64 * c, row0 + 64, fb);
           }
-          for (int j = pc.p0; j < pc.p1; ++j) {
-            if (j + kPrefetchPages < pc.p1) {
-              const int pg = page_of(r, j + kPrefetchPages);
-              if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
-            }
-            int page = page_of(r, j);
-            if (page < 0) {
-              flag_status(p.ws, kStatusBadPage);
-              page = 0;   // any valid page; the consumers mask every token of it
-            }
-            for (int kc = 0; kc < 3; ++kc, ++zc) {
-              const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
-              if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
-              const uint32_t fb = bar(bars->z_full[s]);
-              mbar_arrive_expect_tx(fb, kZStage);
-              const uint32_t dst = sbase + kOffZ + s * kZStage;
-#pragma unroll
-              for (int b = 0; b < 3; ++b) tma_load_3d(dst + b * kBox, &pool_map, 192 * kc + 64 * b, 0, page, fb);
+          for (int j = pc.p0; j < pc.p1; j += 2) {
+            const bool two = j + 1 < pc.p1;
+            for (int u = 0; u < 2; ++u)
+              if (j + u + kPrefetchPages < pc.p1) {
+                const int pg = page_of(r, j + u + kPrefetchPages);
+                if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
+              }
+            int pa = page_of(r, j), pb = two ? page_of(r, j + 1) : 0;
+            if (pa < 0 || pb < 0) flag_status(p.ws, kStatusBadPage);
+            pa = max(pa, 0);     // any valid page; the consumers mask every token of it
+            pb = max(pb, 0);
+            for (int c = 0; c < 9; ++c, ++zc) {
+              uint32_t dst;
+              if (!stage(two ? kZStage : kBox, &dst)) return false;
+              const uint32_t fb = bar(bars->z_full[zc % NZ]);
+              tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
+              if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
             }
           }
           return true;
@@ -314,104 +325,108 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
       }
     } else if (warp == 1) {
-      if (lane == 0) {  // ---- QK^T issuer
-        uint32_t zc = 0, sc = 0, pieces = 0;
+      if (lane == 0) {  // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128)
+        uint32_t zc = 0, bc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
           if (!bwait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
           ++pieces;
-          // the query rows are in TMEM: release their six stages
-          for (int u = 0; u < 6; ++u, ++zc) mbar_arrive(bar(bars->z_empty[zc % NZ]));
+          // the query rows are in TMEM: release their nine stages
+          for (int u = 0; u < 9; ++u, ++zc) mbar_arrive(bar(bars->z_empty[zc % NZ]));
           tc_fence_after();
-          for (int j = pc.p0; j < pc.p1; ++j, ++sc) {
-            const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
-            if (!bwait(ctl, bar(bars->s_empty[sb]), sph ^ 1u)) return false;
-            const uint32_t d = tmem + kTmemS + 64u * sb;
-            for (int kc = 0; kc < 3; ++kc, ++zc) {
-              const uint32_t zs = zc % NZ, zph = (zc / NZ) & 1u;
-              if (!bwait(ctl, bar(bars->z_full[zs]), zph)) return false;
+          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+            if (!bwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
+            for (int c = 0; c < 9; ++c, ++zc) {
+              const uint32_t zs = zc % NZ;
+              if (!bwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
               tc_fence_after();
               const uint32_t za = sbase + kOffZ + zs * kZStage;
 #pragma unroll
-              for (int k = 0; k < 12; ++k) {
-                const int kk = 12 * kc + k;
-                mma_ts(d, tmem + 8u * kk, sdesc(za + (k >> 2) * kBox + (k & 3) * 32, 16, 1024), kIdescQK, kk > 0);
-              }
+              for (int k = 0; k < 4; ++k)
+                mma_ts(tmem + kTmemS, tmem + 8u * (4 * c + k), sdesc(za + 32u * k, 16, 1024), kIdescQK, (c | k) != 0);
               mma_commit(bar(bars->z_empty[zs]));
             }
-            mma_commit(bar(bars->s_full[sb]));
+            mma_commit(bar(bars->s_full));
           }
           return true;
         });
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
-    } else if (warp >= 4 && warp < 8) {
-      // ---- softmax warpgroup: thread i owns row i of the tile (TMEM lane i)
-      const int i = tid - 128, wq = warp - 4;
+    } else if (warp >= 4 && warp < 12) {
+      // ---- softmax: two warpgroups; thread (h, i) owns row i of the tile
+      // (TMEM lane i) for page h of each 2-page block
+      const int g = tid - 128, h = g >> 7, i = g & 127, wq = warp & 3;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
       const uint32_t o_p = mapa(sbase + kOffP, 1);
       const uint32_t o_pfull = mapa(bar(bars->p_full[0]), 1);
       const uint32_t stg = sbase + kOffStage;
-      uint32_t zc = 0, sc = 0, xc = 0;
+      const uint32_t xmax = sbase + kOffXchg, xsum = xmax + 2 * 128 * 4;
+      uint32_t zc = 0, bc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
         const bool valid = rho < rows_total;
         const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
-        // query row i -> TMEM lane i, columns [0, 288) (bf16 pairs).  Rows
-        // 0-63 are in the piece's first three stages, 64-127 in the next
-        // three; every QK MMA of the previous piece has completed because
-        // its last S was read.
+        // query row i -> TMEM lane i, columns [0, 288) (bf16 pairs).  Box c
+        // of the query is stage zc + c (rows 0-63, then 64-127 at +8 KB).
+        // Group 0 moves boxes 0-4, group 1 boxes 5-8.  Every QK MMA of the
+        // previous piece has completed: its last S was read.
         {
-          const int h = i >> 6, ri = i & 63;
+          const uint32_t roff = uint32_t(i >> 6) * kBox + uint32_t(i & 63) * 128;
 #pragma unroll 1
-          for (int kc = 0; kc < 3; ++kc) {
-            const uint32_t idx = zc + 3 * h + kc;
+          for (int c = 0; c < 9; ++c) {
+            const uint32_t idx = zc + c;
             if (!gwait(ctl, bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u)) return false;
-            const uint32_t st = sbase + kOffZ + (idx % NZ) * kZStage + ri * 128;
-#pragma unroll
-            for (int b = 0; b < 3; ++b) {
+            if ((c < 5) == (h == 0)) {
+              const uint32_t st = sbase + kOffZ + (idx % NZ) * kZStage + roff;
               uint32_t v[32];
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
-                const uint4 x = ld_shared_v4(st + b * kBox + ((uint32_t(k) ^ uint32_t(ri & 7)) << 4));
+                const uint4 x = ld_shared_v4(st + ((uint32_t(k) ^ uint32_t(i & 7)) << 4));
                 v[4 * k + 0] = x.x;
                 v[4 * k + 1] = x.y;
                 v[4 * k + 2] = x.z;
                 v[4 * k + 3] = x.w;
               }
-              tmem_st32(tmem + lane_off + 32u * (3 * kc + b), v);
+              tmem_st32(tmem + lane_off + 32u * c, v);
             }
           }
-          zc += 6 + 3 * (pc.p1 - pc.p0);
+          zc += 9 + 9 * ((pc.p1 - pc.p0 + 1) / 2);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
         }
         float m = -INFINITY, l = 0.f;
-        for (int j = pc.p0; j < pc.p1; ++j, ++sc, ++xc) {
-          const uint32_t sb = sc % NS, sph = (sc / NS) & 1u;
-          if (!gwait(ctl, bar(bars->s_full[sb]), sph)) return false;
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          if (!gwait(ctl, bar(bars->s_full), bc & 1u)) return false;
           tc_fence_after();
           uint32_t sv0[32], sv1[32];
-          tmem_ld32(tmem + lane_off + kTmemS + 64u * sb, sv0);
-          tmem_ld32(tmem + lane_off + kTmemS + 64u * sb + 32u, sv1);
+          tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
+          tmem_ld32(tmem + lane_off + kTmemS + 64u * h + 32u, sv1);
           tmem_wait_ld();
           tc_fence_before();
-          mbar_arrive(bar(bars->s_empty[sb]));
+          mbar_arrive(bar(bars->s_empty));
 
-          const int page = p.block_table[size_t(r) * sv.max_pages + j];
-          const bool page_ok = page >= 0 && page < p.num_pages;
-          const int nv = page_ok ? Lrow - j * MLA_PAGE_SIZE : 0;   // visible tokens of this row here
+          const int jp = j + h;                      // this thread's page
+          int nv = 0;                                // its visible tokens here
+          if (jp < pc.p1) {
+            const int page = p.block_table[size_t(r) * sv.max_pages + jp];
+            if (page >= 0 && page < p.num_pages) nv = Lrow - jp * MLA_PAGE_SIZE;
+          }
           float x[64];
-          float mb = -INFINITY;
+          float mh = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             x[c] = c < nv ? __uint_as_float(sv0[c]) * p.scale_log2 : -INFINITY;
             x[c + 32] = c + 32 < nv ? __uint_as_float(sv1[c]) * p.scale_log2 : -INFINITY;
-            mb = fmaxf(mb, fmaxf(x[c], x[c + 32]));
+            mh = fmaxf(mh, fmaxf(x[c], x[c + 32]));
           }
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax + 4u * uint32_t(g)), "f"(mh) : "memory");
+          // staging is free once the previous block's copy has read it
+          if (g == 0) bulk_wait_group_read<0>();
+          named_bar_sync(kSoftmaxBar, kSmThreads);
+          const float mb = fmaxf(mh, ld_shared_f32(xmax + 4u * uint32_t(g ^ 128)));
           float m_new = m, alpha = 1.f;
           bool need = false;
           if (mb > m + kLazyMax) {
@@ -420,40 +435,45 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             need = (j != pc.p0) && (m != -INFINITY);
           }
           const bool live = m_new != -INFINITY;
-          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
-          // staging buffer xs is free once the copy of page xc-2 has read it
-          if (i == 0) bulk_wait_group_read<1>();
-          named_bar_sync(kSoftmaxBar, 128);
-          const uint32_t prow = stg + xs * kPStage + (i >> 3) * 1024 + (i & 7) * 128;
-          float psum = 0.f;
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            float e[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              e[u] = live ? ex2(x[8 * k + u] - m_new) : 0.f;
-              psum += e[u];
-            }
-            st_shared_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(e[0], e[1]), pack_f16(e[2], e[3]),
-                         pack_f16(e[4], e[5]), pack_f16(e[6], e[7]));
+          for (int c = 0; c < 64; c += 4) {
+            x[c] = live ? ex2(x[c] - m_new) : 0.f;
+            x[c + 1] = live ? ex2(x[c + 1] - m_new) : 0.f;
+            x[c + 2] = live ? ex2(x[c + 2] - m_new) : 0.f;
+            x[c + 3] = live ? ex2(x[c + 3] - m_new) : 0.f;
+            s0 += x[c];
+            s1 += x[c + 1];
+            s2 += x[c + 2];
+            s3 += x[c + 3];
           }
-          l = l * alpha + psum;
+          const float ph = (s0 + s1) + (s2 + s3);
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum + 4u * uint32_t(g)), "f"(ph) : "memory");
+          const uint32_t prow = stg + uint32_t(h) * (kPBytes / 2) + (i >> 3) * 1024 + (i & 7) * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(x[8 * k], x[8 * k + 1]),
+                         pack_f16(x[8 * k + 2], x[8 * k + 3]), pack_f16(x[8 * k + 4], x[8 * k + 5]),
+                         pack_f16(x[8 * k + 6], x[8 * k + 7]));
+          named_bar_sync(kSoftmaxBar, kSmThreads);
+          l = l * alpha + ph + ld_shared_f32(xsum + 4u * uint32_t(g ^ 128));
           m = m_new;
-          const uint32_t meta = stg + xs * kPStage + kPBytes;
-          st_shared_u32(meta + 4 * i, __float_as_uint(need ? alpha : 1.f));
-          st_shared_u32(meta + 512 + 4 * i, __float_as_uint(l));
+          if (h == 0) {
+            st_shared_u32(stg + kPBytes + 4 * i, __float_as_uint(need ? alpha : 1.f));
+            st_shared_u32(stg + kPBytes + 512 + 4 * i, __float_as_uint(l));
+          }
           fence_proxy_async_cta();
-          // the output CTA's stage xs is free once PV(xc-2) completed; the
-          // barrier also publishes the staging writes to thread 0
-          const bool free_ok = i == 0 ? bwait(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
-          if (!named_bar_and(kSoftmaxBar, 128, free_ok)) return false;
-          if (i == 0) {
-            mbar_arrive_expect_tx_remote(o_pfull + xs * 8, kPStage);
-            bulk_copy_to_peer(o_p + xs * kPStage, stg + xs * kPStage, kPStage, o_pfull + xs * 8);
+          // the output CTA's block stage is free once its PVs completed;
+          // the barrier also publishes every staging write to thread 0
+          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
+          const bool free_ok = g == 0 ? bwait(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
+          if (!named_bar_and(kSoftmaxBar, kSmThreads, free_ok)) return false;
+          if (g == 0) {
+            bulk_copy_to_peer(o_p + xs * kPStage, stg, kPStage, o_pfull + xs * 8);
             bulk_commit_group();
           }
         }
-        if (valid) {
+        if (valid && h == 0) {
           const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
           if (sv.tile_splits(pc.T) == 1) {
             p.lse[size_t(r) * rows_total + rho] = lse_v;
@@ -466,33 +486,40 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         return true;
       });
       // no copy may still be in flight when the CTAs leave
-      if (i == 0) bulk_wait_group_all();
+      if (g == 0) bulk_wait_group_all();
     }
   } else {
     // ======================= output CTA =======================
     if (warp == 1) {
-      if (lane == 0) {  // ---- PV issuer
-        uint32_t xc = 0, pieces = 0;
+      if (lane == 0) {  // ---- PV issuer: per block, per page 4 K-steps x 2 N halves
+        uint32_t bc = 0, vc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
           if (pieces > 0 && !bwait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
           ++pieces;
-          for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
-            const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
-            if (!bwait(ctl, bar(bars->v_full[xs]), xph)) return false;
-            if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
+          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+            const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
             if (!bwait(ctl, bar(bars->p_full[xs]), xph)) return false;
-            tc_fence_after();
-            const uint32_t pa = sbase + kOffP + xs * kPStage;
-            const uint32_t va = sbase + kOffV + xs * kVStage;
+            if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
+            // arm this stage for its next block (its copy can only start
+            // after this block's PVs complete, which needs corr_done above)
+            mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
+            const int np = min(2, pc.p1 - j);
+            for (int u = 0; u < np; ++u, ++vc) {
+              const uint32_t vs = vc % NV;
+              if (!bwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
+              tc_fence_after();
+              const uint32_t pa = sbase + kOffP + xs * kPStage + uint32_t(u) * (kPBytes / 2);
+              const uint32_t va = sbase + kOffV + vs * kVStage;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t ad = sdesc(pa + 32u * k, 16, 1024);
+              for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = sdesc(pa + 32u * k, 16, 1024);
 #pragma unroll
-              for (int n = 0; n < 2; ++n)
-                mma_ss(tmem + 256u * n, ad, sdesc(va + 4u * n * kBox + 2048u * k, kBox, 1024), kIdescPV,
-                       (j > pc.p0 || k > 0) ? 1u : 0u);
+                for (int n = 0; n < 2; ++n)
+                  mma_ss(tmem + 256u * n, ad, sdesc(va + 4u * n * kBox + 2048u * k, kBox, 1024), kIdescPV,
+                         (j > pc.p0 || u > 0 || k > 0) ? 1u : 0u);
+              }
+              mma_commit(bar(bars->pv_done[vs]));
             }
-            mma_commit(bar(bars->pv_done[xs]));
             mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
           return true;
@@ -504,24 +531,24 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       // ---- correction / epilogue warpgroup: thread i owns row i of O
       const int i = tid - 128, wq = warp - 4;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
-      uint32_t xc = 0;
+      uint32_t bc = 0, vc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
         const bool valid = rho < rows_total;
         float lfin = 0.f;
-        for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
-          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
           if (!wwait(ctl, bar(bars->p_full[xs]), xph)) return false;
           const volatile float* meta = reinterpret_cast<const volatile float*>(gbase + kOffP + xs * kPStage + kPBytes);
           const float alpha = meta[i];
-          if (j == pc.p1 - 1) lfin = meta[128 + i];
+          if (j + 2 >= pc.p1) lfin = meta[128 + i];
           if (__any_sync(0xffffffffu, alpha != 1.f)) {
-            // O must hold every earlier page before it is rescaled.  The
-            // stage's next completion needs this page's corr_done, so the
-            // parity below names PV(page - 1) unambiguously.
-            const uint32_t pv = xc - 1;
-            if (!wwait(ctl, bar(bars->pv_done[pv % NX]), (pv / NX) & 1u)) return false;
+            // O must hold every earlier page before it is rescaled.  That
+            // stage's next completion needs this block's corr_done, so the
+            // parity below names PV(page vc - 1) unambiguously.
+            const uint32_t pv = vc - 1;
+            if (!wwait(ctl, bar(bars->pv_done[pv % NV]), (pv / NV) & 1u)) return false;
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 16; ++c) {
@@ -536,11 +563,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           tc_fence_before();
           mbar_arrive(bar(bars->corr_done[xs]));
+          vc += min(2, pc.p1 - j);
         }
         // epilogue: wait for the last PV, normalise, store
         {
-          const uint32_t pv = xc - 1;
-          if (!wwait(ctl, bar(bars->pv_done[pv % NX]), (pv / NX) & 1u)) return false;
+          const uint32_t pv = vc - 1;
+          if (!wwait(ctl, bar(bars->pv_done[pv % NV]), (pv / NV) & 1u)) return false;
           tc_fence_after();
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
           const bool whole = sv.tile_splits(pc.T) == 1;
@@ -587,7 +615,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       // page's loads are issued right after this page's stores.
       const int ct = tid - 256;
       const int dch = ct & 63, tok0 = ct >> 6;
-      uint32_t xc = 0;
+      uint32_t vc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req;
         const int t = clamp_len(p.seqlens[r], sv);
@@ -604,10 +632,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
         };
         load(pc.p0);
-        for (int j = pc.p0; j < pc.p1; ++j, ++xc) {
-          const uint32_t xs = xc % NX, xph = (xc / NX) & 1u;
-          if (!wwait(ctl, bar(bars->pv_done[xs]), xph ^ 1u)) return false;
-          const uint32_t dst = sbase + kOffV + xs * kVStage + (dch >> 3) * kBox;
+        for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
+          const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
+          if (!wwait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
+          const uint32_t dst = sbase + kOffV + vs * kVStage + (dch >> 3) * kBox;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const int tok = tok0 + 4 * u;
@@ -615,7 +643,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                          bf16x2_to_f16x2(buf[u].y), bf16x2_to_f16x2(buf[u].z), bf16x2_to_f16x2(buf[u].w));
           }
           fence_proxy_async_cta();
-          mbar_arrive(bar(bars->v_full[xs]));
+          mbar_arrive(bar(bars->v_full[vs]));
           if (j + 1 < pc.p1) load(j + 1);
         }
         return true;
