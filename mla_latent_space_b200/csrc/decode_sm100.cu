@@ -56,6 +56,10 @@ using namespace ptx;
 constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring
 constexpr int NX = 2;   // P block stages (output CTA)
 constexpr int NV = 2;   // V page stages (output CTA)
+// Per-block PV completion barriers for the correction warpgroup.  It may lag
+// the MMAs by up to three blocks (a block's P arrives once PV of block - 2
+// completed), so a ring of four keeps every parity wait unambiguous.
+constexpr int NB = 4;
 constexpr int kPrefetchPages = 8;                     // L2 prefetch distance
 constexpr int kThreads = 512;
 constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
@@ -76,7 +80,7 @@ struct Bars {
   // score CTA
   uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
   // output CTA
-  uint64_t v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], o_free;
+  uint64_t v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], pv_blk[NB], o_free;
   // both
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -240,6 +244,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       mbar_init(bar(bars->corr_done[s]), 128);
     }
     for (int s = 0; s < NV; ++s) { mbar_init(bar(bars->v_full[s]), kConvThreads); mbar_init(bar(bars->pv_done[s]), 1); }
+    for (int s = 0; s < NB; ++s) mbar_init(bar(bars->pv_blk[s]), 1);
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
@@ -520,6 +525,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               }
               mma_commit(bar(bars->pv_done[vs]));
             }
+            mma_commit(bar(bars->pv_blk[bc % NB]));
             mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
           return true;
@@ -544,11 +550,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const float alpha = meta[i];
           if (j + 2 >= pc.p1) lfin = meta[128 + i];
           if (__any_sync(0xffffffffu, alpha != 1.f)) {
-            // O must hold every earlier page before it is rescaled.  That
-            // stage's next completion needs this block's corr_done, so the
-            // parity below names PV(page vc - 1) unambiguously.
-            const uint32_t pv = vc - 1;
-            if (!wwait(ctl, bar(bars->pv_done[pv % NV]), (pv / NV) & 1u)) return false;
+            // O must hold every earlier block before it is rescaled (never
+            // the piece's first block, so bc - 1 exists)
+            const uint32_t pb = bc - 1;
+            if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 16; ++c) {
@@ -565,10 +570,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           mbar_arrive(bar(bars->corr_done[xs]));
           vc += min(2, pc.p1 - j);
         }
-        // epilogue: wait for the last PV, normalise, store
+        // epilogue: wait for the piece's last block of PVs, normalise, store
         {
-          const uint32_t pv = vc - 1;
-          if (!wwait(ctl, bar(bars->pv_done[pv % NV]), (pv / NV) & 1u)) return false;
+          const uint32_t pb = bc - 1;
+          if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
           tc_fence_after();
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
           const bool whole = sv.tile_splits(pc.T) == 1;
