@@ -85,6 +85,7 @@ struct Bars {
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort;
+  uint32_t trc[8];   // trace event counters (MLA_TRACE builds)
 };
 
 constexpr uint32_t kOffData = 1024;
@@ -128,7 +129,30 @@ struct Params {
   int num_pages;
   int cap_slots;
   int q_rows;         // batch * s_q * heads
+  unsigned long long* trace;   // event trace (builds with MLA_TRACE only)
 };
+
+// Optional device event trace.  Built only with -DMLA_TRACE: one thread per
+// role of cluster 0 records (event << 24 | index, %globaltimer, clock64)
+// into trace[role][2048][3].  In normal builds the hook compiles to nothing.
+#ifdef MLA_TRACE
+#define MLA_TR(role, ev, j)                                                               \
+  do {                                                                                    \
+    if (p.trace && cluster_id_x() == 0) {                                                 \
+      const unsigned k_ = bars->trc[role]++;                                              \
+      if (k_ < 2048) {                                                                    \
+        unsigned long long* e_ = p.trace + (size_t(role) * 2048 + k_) * 3;                \
+        e_[0] = (unsigned long long)(((ev) << 24) | (unsigned(j) & 0xFFFFFF));            \
+        e_[1] = globaltimer();                                                            \
+        e_[2] = clock64();                                                                \
+      }                                                                                   \
+    }                                                                                     \
+  } while (0)
+#else
+#define MLA_TR(role, ev, j) \
+  do {                      \
+  } while (0)
+#endif
 
 struct Ctl {
   volatile int32_t* abort;
@@ -248,6 +272,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
+    for (int k = 0; k < 8; ++k) bars->trc[k] = 0;
     fence_mbar_init();
     // the output CTA arms its P stages for their first bulk copy
     if (rank == 1)
@@ -281,6 +306,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         auto stage = [&](uint32_t tx, uint32_t* dst) -> bool {
           const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
           if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+          MLA_TR(0, 1, zc);
           mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
           *dst = sbase + kOffZ + s * kZStage;
           return true;
@@ -334,15 +360,18 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         uint32_t zc = 0, bc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
           if (!bwait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
+          MLA_TR(1, 0, bc);
           ++pieces;
           // the query rows are in TMEM: release their nine stages
           for (int u = 0; u < 9; ++u, ++zc) mbar_arrive(bar(bars->z_empty[zc % NZ]));
           tc_fence_after();
           for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
             if (!bwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
+            MLA_TR(1, 2, bc);
             for (int c = 0; c < 9; ++c, ++zc) {
               const uint32_t zs = zc % NZ;
               if (!bwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
+              MLA_TR(1, 10 + c, bc);
               tc_fence_after();
               const uint32_t za = sbase + kOffZ + zs * kZStage;
 #pragma unroll
@@ -351,6 +380,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               mma_commit(bar(bars->z_empty[zs]));
             }
             mma_commit(bar(bars->s_full));
+            MLA_TR(1, 3, bc);
           }
           return true;
         });
@@ -373,6 +403,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         const bool valid = rho < rows_total;
         const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
+        if (g == 0) MLA_TR(2, 9, bc);
         // query row i -> TMEM lane i, columns [0, 288) (bf16 pairs).  Box c
         // of the query is stage zc + c (rows 0-63, then 64-127 at +8 KB).
         // Group 0 moves boxes 0-4, group 1 boxes 5-8.  Every QK MMA of the
@@ -401,10 +432,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
+          if (g == 0) MLA_TR(2, 0, bc);
         }
         float m = -INFINITY, l = 0.f;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
           if (!gwait(ctl, bar(bars->s_full), bc & 1u)) return false;
+          if (g == 0) MLA_TR(2, 1, bc);
           tc_fence_after();
           uint32_t sv0[32], sv1[32];
           tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
@@ -431,6 +464,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           // staging is free once the previous block's copy has read it
           if (g == 0) bulk_wait_group_read<0>();
           named_bar_sync(kSoftmaxBar, kSmThreads);
+          if (g == 0) MLA_TR(2, 5, bc);
           const float mb = fmaxf(mh, ld_shared_f32(xmax + 4u * uint32_t(g ^ 128)));
           float m_new = m, alpha = 1.f;
           bool need = false;
@@ -461,6 +495,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                          pack_f16(x[8 * k + 2], x[8 * k + 3]), pack_f16(x[8 * k + 4], x[8 * k + 5]),
                          pack_f16(x[8 * k + 6], x[8 * k + 7]));
           named_bar_sync(kSoftmaxBar, kSmThreads);
+          if (g == 0) MLA_TR(2, 6, bc);
           l = l * alpha + ph + ld_shared_f32(xsum + 4u * uint32_t(g ^ 128));
           m = m_new;
           if (h == 0) {
@@ -473,9 +508,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
           const bool free_ok = g == 0 ? bwait(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
           if (!named_bar_and(kSoftmaxBar, kSmThreads, free_ok)) return false;
+          if (g == 0) MLA_TR(2, 2, bc);
           if (g == 0) {
             bulk_copy_to_peer(o_p + xs * kPStage, stg, kPStage, o_pfull + xs * 8);
             bulk_commit_group();
+            MLA_TR(2, 3, bc);
           }
         }
         if (valid && h == 0) {
@@ -500,11 +537,14 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         uint32_t bc = 0, vc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
           if (pieces > 0 && !bwait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
+          MLA_TR(4, 0, bc);
           ++pieces;
           for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
             const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
             if (!bwait(ctl, bar(bars->p_full[xs]), xph)) return false;
+            MLA_TR(4, 1, bc);
             if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
+            MLA_TR(4, 2, bc);
             // arm this stage for its next block (its copy can only start
             // after this block's PVs complete, which needs corr_done above)
             mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
@@ -512,6 +552,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             for (int u = 0; u < np; ++u, ++vc) {
               const uint32_t vs = vc % NV;
               if (!bwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
+              MLA_TR(4, 3, vc);
               tc_fence_after();
               const uint32_t pa = sbase + kOffP + xs * kPStage + uint32_t(u) * (kPBytes / 2);
               const uint32_t va = sbase + kOffV + vs * kVStage;
@@ -526,6 +567,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               mma_commit(bar(bars->pv_done[vs]));
             }
             mma_commit(bar(bars->pv_blk[bc % NB]));
+            MLA_TR(4, 4, bc);
             mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
           return true;
@@ -537,7 +579,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       // ---- correction / epilogue warpgroup: thread i owns row i of O
       const int i = tid - 128, wq = warp - 4;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
-      uint32_t bc = 0, vc = 0;
+      uint32_t bc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
@@ -546,6 +588,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
           const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
           if (!wwait(ctl, bar(bars->p_full[xs]), xph)) return false;
+          if (i == 0) MLA_TR(5, 1, bc);
           const volatile float* meta = reinterpret_cast<const volatile float*>(gbase + kOffP + xs * kPStage + kPBytes);
           const float alpha = meta[i];
           if (j + 2 >= pc.p1) lfin = meta[128 + i];
@@ -568,12 +611,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           tc_fence_before();
           mbar_arrive(bar(bars->corr_done[xs]));
-          vc += min(2, pc.p1 - j);
         }
         // epilogue: wait for the piece's last block of PVs, normalise, store
         {
           const uint32_t pb = bc - 1;
           if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
+          if (i == 0) MLA_TR(5, 5, bc);
           tc_fence_after();
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
           const bool whole = sv.tile_splits(pc.T) == 1;
@@ -609,6 +652,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           tc_fence_before();
           mbar_arrive(bar(bars->o_free));
+          if (i == 0) MLA_TR(5, 6, bc);
         }
         return true;
       });
@@ -640,6 +684,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
           const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
           if (!wwait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
+          if (ct == 0) MLA_TR(3, 1, vc);
           const uint32_t dst = sbase + kOffV + vs * kVStage + (dch >> 3) * kBox;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
@@ -649,6 +694,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           fence_proxy_async_cta();
           mbar_arrive(bar(bars->v_full[vs]));
+          if (ct == 0) MLA_TR(3, 3, vc);
           if (j + 1 < pc.p1) load(j + 1);
         }
         return true;
@@ -750,6 +796,7 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   prm.num_pages = shape->num_pages;
   prm.cap_slots = cap_slots;
   prm.q_rows = q_rows;
+  prm.trace = nullptr;
   const int clusters = sms / 2 > 0 ? sms / 2 : 1;
   decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(pool_map, q_map, prm);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
