@@ -167,11 +167,14 @@ __device__ __noinline__ void trip(const Ctl& c) {
 }
 
 // Bounded wait on an mbarrier phase; false when this CTA is aborting.
+// kCluster selects cluster-scope acquire (barriers the peer CTA arrives on).
+template <bool kCluster = false>
 __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_once = [&] { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_once()) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_once()) return true;
     if ((n & 31) == 0) {
       if (*c.abort) return false;
       if (globaltimer() - t0 > kTimeoutNs) {
@@ -184,8 +187,9 @@ __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parit
 
 // Warp-uniform bounded wait: every lane polls, and the warp gives up
 // together if any lane gave up (so no lane is left at a warp collective).
+template <bool kCluster = false>
 __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  const bool ok = bwait(c, bar, parity);
+  const bool ok = bwait<kCluster>(c, bar, parity);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -199,7 +203,7 @@ __device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parit
 // Bounded wait that ignores the abort flag (used while draining).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_cluster(bar, parity)) {
     if (globaltimer() - t0 > kTimeoutNs) return;
   }
 }
@@ -368,11 +372,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
             if (!bwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
             MLA_TR(1, 2, bc);
+            tc_fence_after();
             for (int c = 0; c < 9; ++c, ++zc) {
               const uint32_t zs = zc % NZ;
               if (!bwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
               MLA_TR(1, 10 + c, bc);
-              tc_fence_after();
               const uint32_t za = sbase + kOffZ + zs * kZStage;
 #pragma unroll
               for (int k = 0; k < 4; ++k)
@@ -506,7 +510,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           // the output CTA's block stage is free once its PVs completed;
           // the barrier also publishes every staging write to thread 0
           const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-          const bool free_ok = g == 0 ? bwait(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
+          const bool free_ok = g == 0 ? bwait<true>(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
           if (!named_bar_and(kSoftmaxBar, kSmThreads, free_ok)) return false;
           if (g == 0) MLA_TR(2, 2, bc);
           if (g == 0) {
@@ -541,10 +545,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           ++pieces;
           for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
             const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-            if (!bwait(ctl, bar(bars->p_full[xs]), xph)) return false;
+            if (!bwait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
             MLA_TR(4, 1, bc);
             if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
             MLA_TR(4, 2, bc);
+            tc_fence_after();
             // arm this stage for its next block (its copy can only start
             // after this block's PVs complete, which needs corr_done above)
             mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
@@ -553,7 +558,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               const uint32_t vs = vc % NV;
               if (!bwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
               MLA_TR(4, 3, vc);
-              tc_fence_after();
               const uint32_t pa = sbase + kOffP + xs * kPStage + uint32_t(u) * (kPBytes / 2);
               const uint32_t va = sbase + kOffV + vs * kVStage;
 #pragma unroll
@@ -587,7 +591,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         float lfin = 0.f;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
           const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-          if (!wwait(ctl, bar(bars->p_full[xs]), xph)) return false;
+          if (!wwait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
           if (i == 0) MLA_TR(5, 1, bc);
           const volatile float* meta = reinterpret_cast<const volatile float*>(gbase + kOffP + xs * kPStage + kPBytes);
           const float alpha = meta[i];
