@@ -60,7 +60,11 @@ constexpr int NV = 2;   // V page stages (output CTA)
 // the MMAs by up to three blocks (a block's P arrives once PV of block - 2
 // completed), so a ring of four keeps every parity wait unambiguous.
 constexpr int NB = 4;
-constexpr int kPrefetchPages = 8;                     // L2 prefetch distance
+// L2 bulk-prefetch distance in pages (0 disables the prefetch).
+#ifndef MLA_PREFETCH_PAGES
+#define MLA_PREFETCH_PAGES 8
+#endif
+constexpr int kPrefetchPages = MLA_PREFETCH_PAGES;
 constexpr int kThreads = 512;
 constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
 constexpr uint32_t kZStage = 2 * kBox;                // one 64-column box of both pages (128 rows)
@@ -198,6 +202,16 @@ __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parit
 __device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
   const bool ok = bwait(c, bar, parity);
   return named_bar_and(kSoftmaxBar, kSmThreads, ok);
+}
+
+// Issuer-warp wait: lane 0 polls (it alone issues the tensor-core work that
+// depends on the barrier) and the warp follows its verdict.
+template <bool kCluster = false>
+__device__ __forceinline__ bool lwait(const Ctl& c, uint32_t bar, uint32_t parity, bool leader) {
+  bool ok = true;
+  if (leader) ok = bwait<kCluster>(c, bar, parity);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  return ok;
 }
 
 // Bounded wait that ignores the abort flag (used while draining).
@@ -360,37 +374,54 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
       }
     } else if (warp == 1) {
-      if (lane == 0) {  // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128)
-        uint32_t zc = 0, bc = 0, pieces = 0;
-        each_piece(sv, [&](const Piece& pc) {
-          if (!bwait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
-          MLA_TR(1, 0, bc);
-          ++pieces;
-          // the query rows are in TMEM: release their nine stages
-          for (int u = 0; u < 9; ++u, ++zc) mbar_arrive(bar(bars->z_empty[zc % NZ]));
+      // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128).  The whole
+      // warp runs the loop so every address is warp-uniform; lane 0 issues.
+      // Each stage's descriptor is the ring base's plus a constant step.
+      const bool leader = lane == 0;
+      const uint64_t zdesc0 = sdesc(sbase + kOffZ, 16, 1024);
+      uint32_t zc = 0, bc = 0, pieces = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        if (!lwait(ctl, bar(bars->q_ready), pieces & 1u, leader)) return false;
+        if (leader) MLA_TR(1, 0, bc);
+        ++pieces;
+        // the query rows are in TMEM: release their nine stages
+        if (leader)
+          for (int u = 0; u < 9; ++u) mbar_arrive(bar(bars->z_empty[(zc + u) % NZ]));
+        zc += 9;
+        tc_fence_after();
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          if (!lwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u, leader)) return false;
+          if (leader) MLA_TR(1, 2, bc);
           tc_fence_after();
-          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-            if (!bwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
-            MLA_TR(1, 2, bc);
-            tc_fence_after();
-            for (int c = 0; c < 9; ++c, ++zc) {
-              const uint32_t zs = zc % NZ;
-              if (!bwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
+#pragma unroll 1
+          for (int c = 0; c < 9; ++c, ++zc) {
+            const uint32_t zs = zc % NZ;
+            if (!lwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u, leader)) return false;
+            if (leader) {
               MLA_TR(1, 10 + c, bc);
-              const uint32_t za = sbase + kOffZ + zs * kZStage;
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                mma_ts(tmem + kTmemS, tmem + 8u * (4 * c + k), sdesc(za + 32u * k, 16, 1024), kIdescQK, (c | k) != 0);
+              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
+              mma_ts(d, ad, bd, kIdescQK, c != 0);
+              mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
+              mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
+              mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
               mma_commit(bar(bars->z_empty[zs]));
             }
+            __syncwarp();
+          }
+          if (leader) {
             mma_commit(bar(bars->s_full));
             MLA_TR(1, 3, bc);
           }
-          return true;
-        });
+          __syncwarp();
+        }
+        return true;
+      });
+      if (leader) {
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
+      __syncwarp();
     } else if (warp >= 4 && warp < 12) {
       // ---- softmax: two warpgroups; thread (h, i) owns row i of the tile
       // (TMEM lane i) for page h of each 2-page block
@@ -537,48 +568,60 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   } else {
     // ======================= output CTA =======================
     if (warp == 1) {
-      if (lane == 0) {  // ---- PV issuer: per block, per page 4 K-steps x 2 N halves
-        uint32_t bc = 0, vc = 0, pieces = 0;
-        each_piece(sv, [&](const Piece& pc) {
-          if (pieces > 0 && !bwait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
-          MLA_TR(4, 0, bc);
-          ++pieces;
-          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-            const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-            if (!bwait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
-            MLA_TR(4, 1, bc);
-            if (!bwait(ctl, bar(bars->corr_done[xs]), xph)) return false;
+      // ---- PV issuer: per block, per page 4 K-steps x 2 N halves.  The whole
+      // warp runs the loop (warp-uniform addresses); lane 0 issues.
+      const bool leader = lane == 0;
+      const uint64_t pdesc0 = sdesc(sbase + kOffP, 16, 1024);
+      const uint64_t vdesc0 = sdesc(sbase + kOffV, kBox, 1024);
+      uint32_t bc = 0, vc = 0, pieces = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        if (pieces > 0 && !lwait(ctl, bar(bars->o_free), (pieces - 1) & 1u, leader)) return false;
+        if (leader) MLA_TR(4, 0, bc);
+        ++pieces;
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
+          if (!lwait<true>(ctl, bar(bars->p_full[xs]), xph, leader)) return false;
+          if (leader) MLA_TR(4, 1, bc);
+          if (!lwait(ctl, bar(bars->corr_done[xs]), xph, leader)) return false;
+          if (leader) {
             MLA_TR(4, 2, bc);
-            tc_fence_after();
             // arm this stage for its next block (its copy can only start
             // after this block's PVs complete, which needs corr_done above)
             mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
-            const int np = min(2, pc.p1 - j);
-            for (int u = 0; u < np; ++u, ++vc) {
-              const uint32_t vs = vc % NV;
-              if (!bwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
+          }
+          tc_fence_after();
+          const int np = min(2, pc.p1 - j);
+          for (int u = 0; u < np; ++u, ++vc) {
+            const uint32_t vs = vc % NV;
+            if (!lwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u, leader)) return false;
+            if (leader) {
               MLA_TR(4, 3, vc);
-              const uint32_t pa = sbase + kOffP + xs * kPStage + uint32_t(u) * (kPBytes / 2);
-              const uint32_t va = sbase + kOffV + vs * kVStage;
+              const uint64_t ad = pdesc0 + uint64_t((xs * kPStage + uint32_t(u) * (kPBytes / 2)) >> 4);
+              const uint64_t bd = vdesc0 + uint64_t((vs * kVStage) >> 4);
+              const uint32_t acc0 = (j > pc.p0 || u > 0) ? 1u : 0u;
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = sdesc(pa + 32u * k, 16, 1024);
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-                  mma_ss(tmem + 256u * n, ad, sdesc(va + 4u * n * kBox + 2048u * k, kBox, 1024), kIdescPV,
-                         (j > pc.p0 || u > 0 || k > 0) ? 1u : 0u);
+                mma_ss(tmem, ad + 2u * k, bd + (2048u >> 4) * k, kIdescPV, k > 0 ? 1u : acc0);
+                mma_ss(tmem + 256u, ad + 2u * k, bd + ((4u * kBox + 2048u * k) >> 4), kIdescPV, k > 0 ? 1u : acc0);
               }
               mma_commit(bar(bars->pv_done[vs]));
             }
+            __syncwarp();
+          }
+          if (leader) {
             mma_commit(bar(bars->pv_blk[bc % NB]));
             MLA_TR(4, 4, bc);
             mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
-          return true;
-        });
+          __syncwarp();
+        }
+        return true;
+      });
+      if (leader) {
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
+      __syncwarp();
     } else if (warp >= 4 && warp < 8) {
       // ---- correction / epilogue warpgroup: thread i owns row i of O
       const int i = tid - 128, wq = warp - 4;
