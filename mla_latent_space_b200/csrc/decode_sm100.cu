@@ -62,7 +62,7 @@ constexpr int NV = 2;   // V page stages (output CTA)
 constexpr int NB = 4;
 // L2 bulk-prefetch distance in pages (0 disables the prefetch).
 #ifndef MLA_PREFETCH_PAGES
-#define MLA_PREFETCH_PAGES 8
+#define MLA_PREFETCH_PAGES 0
 #endif
 constexpr int kPrefetchPages = MLA_PREFETCH_PAGES;
 constexpr int kThreads = 512;
@@ -179,7 +179,10 @@ __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parit
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
     if (try_once()) return true;
-    if ((n & 31) == 0) {
+    // back off after a few misses so that waiting warps leave the issue
+    // slots to the warps doing the work
+    if (n > 4) __nanosleep(n > 64 ? 256 : 32);
+    if ((n & 15) == 0) {
       if (*c.abort) return false;
       if (globaltimer() - t0 > kTimeoutNs) {
         trip(c);
@@ -189,18 +192,22 @@ __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parit
   }
 }
 
-// Warp-uniform bounded wait: every lane polls, and the warp gives up
-// together if any lane gave up (so no lane is left at a warp collective).
+// Warp-uniform bounded wait: lane 0 polls, the warp follows its verdict.
+// __syncwarp orders the other lanes' later accesses after lane 0's acquire.
 template <bool kCluster = false>
 __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  const bool ok = bwait<kCluster>(c, bar, parity);
-  return __all_sync(0xffffffffu, ok);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = bwait<kCluster>(c, bar, parity);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
 }
 
 // Softmax-group bounded wait: the 256 threads decide together (a thread
 // leaving alone would strand the others at the group's named barrier).
 __device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  const bool ok = bwait(c, bar, parity);
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = bwait(c, bar, parity);
   return named_bar_and(kSoftmaxBar, kSmThreads, ok);
 }
 
@@ -211,6 +218,7 @@ __device__ __forceinline__ bool lwait(const Ctl& c, uint32_t bar, uint32_t parit
   bool ok = true;
   if (leader) ok = bwait<kCluster>(c, bar, parity);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
   return ok;
 }
 
@@ -348,7 +356,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           for (int j = pc.p0; j < pc.p1; j += 2) {
             const bool two = j + 1 < pc.p1;
             for (int u = 0; u < 2; ++u)
-              if (j + u + kPrefetchPages < pc.p1) {
+              if (kPrefetchPages > 0 && j + u + kPrefetchPages < pc.p1) {
                 const int pg = page_of(r, j + u + kPrefetchPages);
                 if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
               }
