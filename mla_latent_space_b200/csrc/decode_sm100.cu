@@ -23,11 +23,12 @@
 //     They write P (fp16, in the output CTA's swizzled layout) and per-row
 //     rescale factors to a staging buffer, which one thread ships to the
 //     output CTA with a single bulk copy over distributed shared memory.
-//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  Eight converter
-//     warps read each page's 512 value columns from global memory (L2, where
-//     CTA 0 prefetched them), convert bf16 -> fp16 (exact in fp16's normal
-//     range) and store them in the 128-byte swizzled N-major layout, the next
-//     page's loads in flight during the store.  One thread issues
+//   CTA 1 ("output"): O (128 x 512 fp32) fills its TMEM.  Its own TMA warp
+//     streams each page's 512 value columns (8 boxes, 128-byte swizzle, which
+//     is the N-major operand layout) through a 3-deep ring; eight converter
+//     warps rewrite each landed stage in place from bf16 to fp16 (exact in
+//     fp16's normal range).  Each SM ingests at most ~60 GB/s, so both CTAs
+//     keep ~190 KB of loads in flight.  One thread issues
 //     O += P . V (M=128, N=256, K=16, twice per 16 tokens) page by page; a
 //     warpgroup applies the rare rescales to O between blocks and writes the
 //     normalised result at the end of a piece.
@@ -54,8 +55,8 @@ namespace {
 using namespace ptx;
 
 constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring
-constexpr int NX = 2;   // P block stages (output CTA)
-constexpr int NV = 2;   // V page stages (output CTA)
+constexpr int NX = 1;   // P block stages (output CTA)
+constexpr int NV = 3;   // V page stages (output CTA): its own TMA ring
 // Per-block PV completion barriers for the correction warpgroup.  It may lag
 // the MMAs by up to three blocks (a block's P arrives once PV of block - 2
 // completed), so a ring of four keeps every parity wait unambiguous.
@@ -84,7 +85,7 @@ struct Bars {
   // score CTA
   uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
   // output CTA
-  uint64_t v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], pv_blk[NB], o_free;
+  uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], pv_blk[NB], o_free;
   // both
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -293,7 +294,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       mbar_init(bar(bars->p_full[s]), 1);
       mbar_init(bar(bars->corr_done[s]), 128);
     }
-    for (int s = 0; s < NV; ++s) { mbar_init(bar(bars->v_full[s]), kConvThreads); mbar_init(bar(bars->pv_done[s]), 1); }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(bar(bars->v_loaded[s]), 1);
+      mbar_init(bar(bars->v_full[s]), kConvThreads);
+      mbar_init(bar(bars->pv_done[s]), 1);
+    }
     for (int s = 0; s < NB; ++s) mbar_init(bar(bars->pv_blk[s]), 1);
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
@@ -304,9 +309,9 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     if (rank == 1)
       for (int s = 0; s < NX; ++s) mbar_arrive_expect_tx(bar(bars->p_full[s]), kPStage);
   }
-  if (warp == 0 && lane == 0 && rank == 0) {
+  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&pool_map);
-    tma_prefetch_desc(&q_map);
+    if (rank == 0) tma_prefetch_desc(&q_map);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
@@ -711,46 +716,62 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
         return true;
       });
+    } else if (warp == 0) {
+      if (lane == 0) {  // ---- V producer: the page's first 512 columns (8 boxes) per stage
+        uint32_t vc = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          const int r = pc.T / sv.tiles_per_req;
+          for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
+            const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
+            if (!bwait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
+            int page = p.block_table[size_t(r) * sv.max_pages + j];
+            if (page < 0 || page >= p.num_pages) page = 0;   // the converters zero it
+            const uint32_t fb = bar(bars->v_loaded[vs]);
+            mbar_arrive_expect_tx(fb, kVStage);
+            const uint32_t dst = sbase + kOffV + vs * kVStage;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) tma_load_3d(dst + c * kBox, &pool_map, 64 * c, 0, page, fb);
+          }
+          return true;
+        });
+        const uint32_t n = vc < NV ? vc : NV;
+        for (uint32_t k = 1; k <= n; ++k) {
+          const uint32_t idx = vc - k;
+          drain_wait(bar(bars->v_loaded[idx % NV]), (idx / NV) & 1u);
+        }
+      }
     } else if (warp >= 8) {
-      // ---- V converters: thread -> one 16-byte column chunk (8 values) of
-      // 16 of the page's 64 tokens.  Global bf16 -> fp16 -> the swizzled
-      // N-major stage.  Tokens at or past the request's length are zero
-      // (their bytes may be anything; 0 * NaN would poison O).  The next
-      // page's loads are issued right after this page's stores.
+      // ---- V converters: each landed stage is rewritten in place from bf16
+      // to fp16 (same size, same swizzled N-major layout).  Tokens at or
+      // past the request's length become zero: their bytes may be anything
+      // and 0 * NaN would poison O.  Thread -> 16 chunks of 16 bytes.
       const int ct = tid - 256;
-      const int dch = ct & 63, tok0 = ct >> 6;
       uint32_t vc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req;
         const int t = clamp_len(p.seqlens[r], sv);
-        uint4 buf[16];
-        auto load = [&](int j) {
+        for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
+          const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
           const int page = p.block_table[size_t(r) * sv.max_pages + j];
           const bool ok = page >= 0 && page < p.num_pages;
           const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
-          const uint8_t* src = p.kv + size_t(ok ? page : 0) * kPageBytes + dch * 16;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int tok = tok0 + 4 * u;
-            buf[u] = tok < nvalid ? ld_global_nc_v4(src + size_t(tok) * (MLA_D_QK * 2)) : make_uint4(0, 0, 0, 0);
-          }
-        };
-        load(pc.p0);
-        for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
-          const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
-          if (!wwait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
+          if (!wwait(ctl, bar(bars->v_loaded[vs]), vph)) return false;
           if (ct == 0) MLA_TR(3, 1, vc);
-          const uint32_t dst = sbase + kOffV + vs * kVStage + (dch >> 3) * kBox;
+          const uint32_t st = sbase + kOffV + vs * kVStage;
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            const int tok = tok0 + 4 * u;
-            st_shared_v4(dst + tok * 128 + ((uint32_t(dch & 7) ^ uint32_t(tok & 7)) << 4), bf16x2_to_f16x2(buf[u].x),
-                         bf16x2_to_f16x2(buf[u].y), bf16x2_to_f16x2(buf[u].z), bf16x2_to_f16x2(buf[u].w));
+            const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
+            const int tok = int((off & (kBox - 1)) >> 7);
+            const uint4 v = ld_shared_v4(st + off);
+            if (tok < nvalid)
+              st_shared_v4(st + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                           bf16x2_to_f16x2(v.w));
+            else
+              st_shared_v4(st + off, 0u, 0u, 0u, 0u);
           }
           fence_proxy_async_cta();
           mbar_arrive(bar(bars->v_full[vs]));
           if (ct == 0) MLA_TR(3, 3, vc);
-          if (j + 1 < pc.p1) load(j + 1);
         }
         return true;
       });
