@@ -138,8 +138,12 @@ struct Params {
 };
 
 // Optional device event trace.  Built only with -DMLA_TRACE: one thread per
-// role of cluster 0 records (event << 24 | index, %globaltimer, clock64)
-// into trace[role][2048][3].  In normal builds the hook compiles to nothing.
+// role of cluster 0 records (event << 24 | index, clock64, 0) into
+// trace[role][2048][3]; roles 6 and 7 hold one (0, clock64, %globaltimer)
+// pair per CTA taken right after the start-up cluster barrier, to line the
+// two SMs' clocks up.  Only the SM clock is read per event (the global timer
+// is far slower to read and would distort the timeline).  In normal builds
+// the hooks compile to nothing.
 #ifdef MLA_TRACE
 #define MLA_TR(role, ev, j)                                                               \
   do {                                                                                    \
@@ -148,14 +152,24 @@ struct Params {
       if (k_ < 2048) {                                                                    \
         unsigned long long* e_ = p.trace + (size_t(role) * 2048 + k_) * 3;                \
         e_[0] = (unsigned long long)(((ev) << 24) | (unsigned(j) & 0xFFFFFF));            \
-        e_[1] = globaltimer();                                                            \
-        e_[2] = clock64();                                                                \
+        e_[1] = clock64();                                                                \
       }                                                                                   \
+    }                                                                                     \
+  } while (0)
+#define MLA_TR_SYNC(role)                                                                 \
+  do {                                                                                    \
+    if (p.trace && cluster_id_x() == 0) {                                                 \
+      unsigned long long* e_ = p.trace + size_t(role) * 2048 * 3;                         \
+      e_[1] = clock64();                                                                  \
+      e_[2] = globaltimer();                                                              \
     }                                                                                     \
   } while (0)
 #else
 #define MLA_TR(role, ev, j) \
   do {                      \
+  } while (0)
+#define MLA_TR_SYNC(role) \
+  do {                    \
   } while (0)
 #endif
 
@@ -173,16 +187,19 @@ __device__ __noinline__ void trip(const Ctl& c) {
 
 // Bounded wait on an mbarrier phase; false when this CTA is aborting.
 // kCluster selects cluster-scope acquire (barriers the peer CTA arrives on).
-template <bool kCluster = false>
+// kSpin polls with test_wait (no suspension: for the single threads that
+// feed the tensor core and the copy engine); otherwise try_wait, which lets
+// the hardware suspend a waiting warp between polls.
+template <bool kCluster = false, bool kSpin = false>
 __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parity) {
-  auto try_once = [&] { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  auto try_once = [&] {
+    if (kSpin) return kCluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity);
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
   if (try_once()) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
     if (try_once()) return true;
-    // back off after a few misses so that waiting warps leave the issue
-    // slots to the warps doing the work
-    if (n > 4) __nanosleep(n > 64 ? 256 : 32);
     if ((n & 15) == 0) {
       if (*c.abort) return false;
       if (globaltimer() - t0 > kTimeoutNs) {
@@ -191,6 +208,12 @@ __device__ __forceinline__ bool bwait(const Ctl& c, uint32_t bar, uint32_t parit
       }
     }
   }
+}
+
+// Pipeline-driver wait: a spinning bwait.
+template <bool kCluster = false>
+__device__ __forceinline__ bool swait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  return bwait<kCluster, true>(c, bar, parity);
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the warp follows its verdict.
@@ -204,23 +227,14 @@ __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parit
   return ok;
 }
 
-// Softmax-group bounded wait: the 256 threads decide together (a thread
-// leaving alone would strand the others at the group's named barrier).
-__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity) {
+// Softmax-group bounded wait: the group's first thread polls, the named
+// barrier hands its verdict (and, through the barrier, its acquire) to the
+// other 255 threads, and the group decides together (a thread leaving alone
+// would strand the others at the group's named barrier).
+__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity, bool poller) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = bwait(c, bar, parity);
+  if (poller) ok = bwait(c, bar, parity);
   return named_bar_and(kSoftmaxBar, kSmThreads, ok);
-}
-
-// Issuer-warp wait: lane 0 polls (it alone issues the tensor-core work that
-// depends on the barrier) and the warp follows its verdict.
-template <bool kCluster = false>
-__device__ __forceinline__ bool lwait(const Ctl& c, uint32_t bar, uint32_t parity, bool leader) {
-  bool ok = true;
-  if (leader) ok = bwait<kCluster>(c, bar, parity);
-  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  __syncwarp();
-  return ok;
 }
 
 // Bounded wait that ignores the abort flag (used while draining).
@@ -324,6 +338,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   cluster_sync();
 
   Ctl ctl{&bars->abort, mapa(smem_u32(&bars->abort), rank ^ 1u), p.ws};
+  if (tid == 0) MLA_TR_SYNC(6 + rank);
 
   if (rank == 0) {
     // ======================= score CTA =======================
@@ -336,7 +351,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         };
         auto stage = [&](uint32_t tx, uint32_t* dst) -> bool {
           const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
-          if (!bwait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+          if (!swait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
           MLA_TR(0, 1, zc);
           mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
           *dst = sbase + kOffZ + s * kZStage;
@@ -387,30 +402,24 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
       }
     } else if (warp == 1) {
-      // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128).  The whole
-      // warp runs the loop so every address is warp-uniform; lane 0 issues.
-      // Each stage's descriptor is the ring base's plus a constant step.
-      const bool leader = lane == 0;
-      const uint64_t zdesc0 = sdesc(sbase + kOffZ, 16, 1024);
-      uint32_t zc = 0, bc = 0, pieces = 0;
-      each_piece(sv, [&](const Piece& pc) {
-        if (!lwait(ctl, bar(bars->q_ready), pieces & 1u, leader)) return false;
-        if (leader) MLA_TR(1, 0, bc);
-        ++pieces;
-        // the query rows are in TMEM: release their nine stages
-        if (leader)
+      if (lane == 0) {  // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128)
+        const uint64_t zdesc0 = sdesc(sbase + kOffZ, 16, 1024);
+        uint32_t zc = 0, bc = 0, pieces = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          if (!swait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
+          MLA_TR(1, 0, bc);
+          ++pieces;
+          // the query rows are in TMEM: release their nine stages
           for (int u = 0; u < 9; ++u) mbar_arrive(bar(bars->z_empty[(zc + u) % NZ]));
-        zc += 9;
-        tc_fence_after();
-        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-          if (!lwait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u, leader)) return false;
-          if (leader) MLA_TR(1, 2, bc);
+          zc += 9;
           tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 9; ++c, ++zc) {
-            const uint32_t zs = zc % NZ;
-            if (!lwait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u, leader)) return false;
-            if (leader) {
+          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+            if (!swait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
+            MLA_TR(1, 2, bc);
+            tc_fence_after();
+            for (int c = 0; c < 9; ++c, ++zc) {
+              const uint32_t zs = zc % NZ;
+              if (!swait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
               MLA_TR(1, 10 + c, bc);
               const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
               const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
@@ -420,21 +429,14 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
               mma_commit(bar(bars->z_empty[zs]));
             }
-            __syncwarp();
-          }
-          if (leader) {
             mma_commit(bar(bars->s_full));
             MLA_TR(1, 3, bc);
           }
-          __syncwarp();
-        }
-        return true;
-      });
-      if (leader) {
+          return true;
+        });
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
-      __syncwarp();
     } else if (warp >= 4 && warp < 12) {
       // ---- softmax: two warpgroups; thread (h, i) owns row i of the tile
       // (TMEM lane i) for page h of each 2-page block
@@ -461,7 +463,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 #pragma unroll 1
           for (int c = 0; c < 9; ++c) {
             const uint32_t idx = zc + c;
-            if (!gwait(ctl, bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u)) return false;
+            if (!gwait(ctl, bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u, g == 0)) return false;
             if ((c < 5) == (h == 0)) {
               const uint32_t st = sbase + kOffZ + (idx % NZ) * kZStage + roff;
               uint32_t v[32];
@@ -484,7 +486,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
         float m = -INFINITY, l = 0.f;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-          if (!gwait(ctl, bar(bars->s_full), bc & 1u)) return false;
+          if (!gwait(ctl, bar(bars->s_full), bc & 1u, g == 0)) return false;
           if (g == 0) MLA_TR(2, 1, bc);
           tc_fence_after();
           uint32_t sv0[32], sv1[32];
@@ -581,33 +583,28 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   } else {
     // ======================= output CTA =======================
     if (warp == 1) {
-      // ---- PV issuer: per block, per page 4 K-steps x 2 N halves.  The whole
-      // warp runs the loop (warp-uniform addresses); lane 0 issues.
-      const bool leader = lane == 0;
-      const uint64_t pdesc0 = sdesc(sbase + kOffP, 16, 1024);
-      const uint64_t vdesc0 = sdesc(sbase + kOffV, kBox, 1024);
-      uint32_t bc = 0, vc = 0, pieces = 0;
-      each_piece(sv, [&](const Piece& pc) {
-        if (pieces > 0 && !lwait(ctl, bar(bars->o_free), (pieces - 1) & 1u, leader)) return false;
-        if (leader) MLA_TR(4, 0, bc);
-        ++pieces;
-        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-          if (!lwait<true>(ctl, bar(bars->p_full[xs]), xph, leader)) return false;
-          if (leader) MLA_TR(4, 1, bc);
-          if (!lwait(ctl, bar(bars->corr_done[xs]), xph, leader)) return false;
-          if (leader) {
+      if (lane == 0) {  // ---- PV issuer: per block, per page 4 K-steps x 2 N halves
+        const uint64_t pdesc0 = sdesc(sbase + kOffP, 16, 1024);
+        const uint64_t vdesc0 = sdesc(sbase + kOffV, kBox, 1024);
+        uint32_t bc = 0, vc = 0, pieces = 0;
+        each_piece(sv, [&](const Piece& pc) {
+          if (pieces > 0 && !swait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
+          MLA_TR(4, 0, bc);
+          ++pieces;
+          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+            const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
+            if (!swait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
+            MLA_TR(4, 1, bc);
+            if (!swait(ctl, bar(bars->corr_done[xs]), xph)) return false;
             MLA_TR(4, 2, bc);
             // arm this stage for its next block (its copy can only start
             // after this block's PVs complete, which needs corr_done above)
             mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
-          }
-          tc_fence_after();
-          const int np = min(2, pc.p1 - j);
-          for (int u = 0; u < np; ++u, ++vc) {
-            const uint32_t vs = vc % NV;
-            if (!lwait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u, leader)) return false;
-            if (leader) {
+            tc_fence_after();
+            const int np = min(2, pc.p1 - j);
+            for (int u = 0; u < np; ++u, ++vc) {
+              const uint32_t vs = vc % NV;
+              if (!swait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
               MLA_TR(4, 3, vc);
               const uint64_t ad = pdesc0 + uint64_t((xs * kPStage + uint32_t(u) * (kPBytes / 2)) >> 4);
               const uint64_t bd = vdesc0 + uint64_t((vs * kVStage) >> 4);
@@ -619,22 +616,15 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               }
               mma_commit(bar(bars->pv_done[vs]));
             }
-            __syncwarp();
-          }
-          if (leader) {
             mma_commit(bar(bars->pv_blk[bc % NB]));
             MLA_TR(4, 4, bc);
             mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
-          __syncwarp();
-        }
-        return true;
-      });
-      if (leader) {
+          return true;
+        });
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
-      __syncwarp();
     } else if (warp >= 4 && warp < 8) {
       // ---- correction / epilogue warpgroup: thread i owns row i of O
       const int i = tid - 128, wq = warp - 4;
@@ -723,7 +713,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const int r = pc.T / sv.tiles_per_req;
           for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
             const uint32_t vs = vc % NV, vph = (vc / NV) & 1u;
-            if (!bwait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
+            if (!swait(ctl, bar(bars->pv_done[vs]), vph ^ 1u)) return false;
             int page = p.block_table[size_t(r) * sv.max_pages + j];
             if (page < 0 || page >= p.num_pages) page = 0;   // the converters zero it
             const uint32_t fb = bar(bars->v_loaded[vs]);
