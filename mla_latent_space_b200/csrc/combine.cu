@@ -4,10 +4,13 @@
 // Tiles that no worker touched (no visible key) get O = 0 and lse = -inf.
 //
 // One warp per row, (tile, 16 row blocks) CTAs of 8 warps: the lanes read
-// the pieces' lse values at once, reduce max and sum with shuffles, then
-// stream the 512 fp32 values of up to four pieces per round with float4
-// loads all in flight together.
+// the pieces' lse values at once and reduce max and sum with shuffles; then
+// each lane streams its 16 fp32 values of one piece at a time (four float4
+// loads in flight per lane).  At most 64 registers a thread, so that four
+// CTAs share an SM and every row of a typical batch is in flight in about
+// one wave: the kernel is bound by how many loads are outstanding.
 #include "kernel_util.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 
@@ -16,9 +19,10 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kRowBlocks = MLA_TILE_ROWS / kWarps;   // 16
 
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 4)
 combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __nv_bfloat16* __restrict__ out,
                float* __restrict__ lse, int cap_slots) {
+  ptx::griddep_wait();   // launched programmatically behind the decode kernel
   const SchedView sv(sched);
   void* ws = const_cast<void*>(ws_c);
   const int T = blockIdx.x;
@@ -42,6 +46,14 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
     if (lane == 0) lse[size_t(r) * rows_total + rho] = -INFINITY;
     return;
   }
+  // the first piece's values do not depend on the weights: their loads go
+  // out before the lse reduction so that the two latencies overlap
+  float4 v0[MLA_D_V / 128];
+  {
+    const float4* src = reinterpret_cast<const float4*>(ws_partial_o(ws, cap_slots, base) + size_t(row) * MLA_D_V);
+#pragma unroll
+    for (int c = 0; c < MLA_D_V / 128; ++c) v0[c] = __ldcs(src + lane + 32 * c);
+  }
   float mx = -INFINITY;
   for (int i = lane; i < n; i += 32) mx = fmaxf(mx, ws_partial_lse(ws, cap_slots, base + i)[row]);
 #pragma unroll
@@ -56,31 +68,25 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
 #pragma unroll
   for (int c = 0; c < MLA_D_V / 128; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (L != -INFINITY) {
-    for (int i0 = 0; i0 < n; i0 += 4) {
-      float4 v[4][MLA_D_V / 128];
-      float w[4];
+    for (int i = 0; i < n; ++i) {
+      const float w = __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - L);
+      float4 v[MLA_D_V / 128];
+      if (i == 0) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = i0 + k;
-        w[k] = 0.f;
-        if (i < n) {
-          w[k] = __expf(ws_partial_lse(ws, cap_slots, base + i)[row] - L);
-          const float4* src =
-              reinterpret_cast<const float4*>(ws_partial_o(ws, cap_slots, base + i) + size_t(row) * MLA_D_V);
+        for (int c = 0; c < MLA_D_V / 128; ++c) v[c] = v0[c];
+      } else {
+        const float4* src =
+            reinterpret_cast<const float4*>(ws_partial_o(ws, cap_slots, base + i) + size_t(row) * MLA_D_V);
 #pragma unroll
-          for (int c = 0; c < MLA_D_V / 128; ++c) v[k][c] = __ldcs(src + lane + 32 * c);
-        }
+        for (int c = 0; c < MLA_D_V / 128; ++c) v[c] = __ldcs(src + lane + 32 * c);
       }
+      if (w == 0.f) continue;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (w[k] == 0.f) continue;
-#pragma unroll
-        for (int c = 0; c < MLA_D_V / 128; ++c) {
-          acc[c].x = fmaf(w[k], v[k][c].x, acc[c].x);
-          acc[c].y = fmaf(w[k], v[k][c].y, acc[c].y);
-          acc[c].z = fmaf(w[k], v[k][c].z, acc[c].z);
-          acc[c].w = fmaf(w[k], v[k][c].w, acc[c].w);
-        }
+      for (int c = 0; c < MLA_D_V / 128; ++c) {
+        acc[c].x = fmaf(w, v[c].x, acc[c].x);
+        acc[c].y = fmaf(w, v[c].y, acc[c].y);
+        acc[c].z = fmaf(w, v[c].z, acc[c].z);
+        acc[c].w = fmaf(w, v[c].w, acc[c].w);
       }
     }
   }
@@ -101,9 +107,21 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
 cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
                            int cap_slots, cudaStream_t stream) {
   if (num_tiles == 0) return cudaSuccess;
-  combine_kernel<<<dim3(num_tiles, kRowBlocks), kWarps * 32, 0, stream>>>(
-      sched, ws, static_cast<__nv_bfloat16*>(out), lse, cap_slots);
-  return cudaGetLastError();
+  // programmatic dependent launch behind the decode kernel (the kernel waits
+  // for it before reading anything)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_tiles, kRowBlocks);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, sched, ws, static_cast<__nv_bfloat16*>(out), lse,
+                                           cap_slots);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace mla

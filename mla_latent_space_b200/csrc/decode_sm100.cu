@@ -295,8 +295,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-  const SchedView sv(p.sched);
-  const int rows_total = sv.s_q * sv.heads;
 
   if (tid == 0) {
     for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
@@ -336,6 +334,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   cluster_sync();
+  // everything above overlaps the scheduler kernel still running before us
+  // (programmatic dependent launch); its schedule is read from here on
+  griddep_wait();
+  griddep_launch_dependents();
+  const SchedView sv(p.sched);
+  const int rows_total = sv.s_q * sv.heads;
 
   Ctl ctl{&bars->abort, mapa(smem_u32(&bars->abort), rank ^ 1u), p.ws};
   if (tid == 0) MLA_TR_SYNC(6 + rank);
@@ -864,8 +868,21 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   prm.q_rows = q_rows;
   prm.trace = nullptr;
   const int clusters = sms / 2 > 0 ? sms / 2 : 1;
-  decode_sm100_kernel<<<2 * clusters, kThreads, kSmemBytes, stream>>>(pool_map, q_map, prm);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  // programmatic dependent launch: the prologue (barriers, TMEM, descriptor
+  // prefetch) overlaps the scheduler kernel; the kernel waits for it before
+  // reading the schedule
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_sm100_kernel, pool_map, q_map, prm);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace mla

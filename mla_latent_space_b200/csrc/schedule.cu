@@ -70,102 +70,137 @@ MLA_HD void worker_start(const int32_t* tiles, int num_tiles, int64_t total, int
   map_position(tiles, num_tiles, total * w / We, tile, page);
 }
 
-constexpr int kSchedThreads = 1024;
+// ---- device scheduler ------------------------------------------------------
+// One CTA.  The tile costs, their prefix and the worker start keys live in
+// shared memory, so that the binary searches of the position mapping (a few
+// dozen dependent lookups) never wait on global memory; only the results go
+// out.  Schedules too large for shared memory take the same steps on the
+// global copies (schedule_kernel_global).
+constexpr int kSchedThreads = 256;
+constexpr int kSchedWarps = kSchedThreads / 32;
+constexpr size_t kSchedSmemMax = 200 * 1024;
 
-// Block-wide exclusive scan of one int64 per thread; returns the total.
-__device__ int64_t block_exclusive_scan(int64_t v, int64_t* buf, int64_t* excl) {
-  int tid = threadIdx.x;
-  buf[tid] = v;
-  __syncthreads();
-  for (int off = 1; off < kSchedThreads; off <<= 1) {
-    int64_t add = tid >= off ? buf[tid - off] : 0;
-    __syncthreads();
-    buf[tid] += add;
-    __syncthreads();
+// Block-wide exclusive scan of one int64 per thread (warp shuffles, then the
+// warp totals); returns the block total.
+__device__ int64_t block_exclusive_scan(int64_t v, int64_t* warp_tot, int64_t* excl) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int64_t inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int64_t u = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += u;
   }
-  *excl = buf[tid] - v;
-  int64_t total = buf[kSchedThreads - 1];
+  if (lane == 31) warp_tot[warp] = inc;
   __syncthreads();
+  int64_t base = 0, total = 0;
+#pragma unroll
+  for (int k = 0; k < kSchedWarps; ++k) {
+    const int64_t t = warp_tot[k];
+    base += k < warp ? t : 0;
+    total += t;
+  }
+  *excl = base + inc - v;
+  __syncthreads();   // warp_tot may be reused by the next scan
   return total;
+}
+
+// First index in [0, W) whose key is >= key (keys non-decreasing).
+__device__ __forceinline__ int first_key_ge(const int64_t* keys, int W, int64_t key) {
+  int lo = 0, hi = W;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (keys[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// Shared-memory layout: pages[num_tiles], prefix[num_tiles] (int32), then
+// wkey[W] (int64, 8-byte aligned).
+MLA_HD size_t sched_smem_bytes(int num_tiles, int W) {
+  return ((size_t(num_tiles) * 8 + 7) & ~size_t(7)) + size_t(W) * 8;
 }
 
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t* __restrict__ sched) {
-  __shared__ int64_t buf[kSchedThreads];
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int64_t warp_tot[kSchedWarps];
   __shared__ int32_t flag_sh;
-  int tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int num_tiles = s.batch * s.tiles_per_req;
+  int32_t* pages_sm = reinterpret_cast<int32_t*>(smem);
+  int32_t* prefix_sm = pages_sm + num_tiles;
+  int64_t* wkey = reinterpret_cast<int64_t*>(smem + ((size_t(num_tiles) * 8 + 7) & ~size_t(7)));
   int32_t* hdr = sched;
   int32_t* workers = sched + kHeaderInts;
   int32_t* tiles = workers + size_t(W) * kWorkerInts;
   if (tid == 0) flag_sh = 0;
   __syncthreads();
 
-  // 1-2: tile pages, costs and their exclusive prefix
+  // 1-2: tile pages, costs and their exclusive prefix (contiguous chunks)
   const int chunk = (num_tiles + kSchedThreads - 1) / kSchedThreads;
-  const int t0 = tid * chunk, t1 = min(num_tiles, t0 + chunk);
+  const int t0 = min(num_tiles, tid * chunk), t1 = min(num_tiles, t0 + chunk);
   int32_t flag = 0;
   int64_t local = 0;
   for (int T = t0; T < t1; ++T) {
-    int r = T / s.tiles_per_req, qt = T % s.tiles_per_req;
-    int t = clamp_seqlen(seqlens[r], s.max_pages, &flag);
-    int pages = tile_pages(s, t, qt);
-    tiles[size_t(T) * kTileInts + T_PAGES] = pages;
+    const int r = T / s.tiles_per_req, qt = T % s.tiles_per_req;
+    const int t = clamp_seqlen(seqlens[r], s.max_pages, &flag);
+    const int pages = tile_pages(s, t, qt);
+    pages_sm[T] = pages;
     local += tile_cost(pages);
   }
   if (flag) atomicOr(&flag_sh, flag);
   int64_t excl;
-  const int64_t total = block_exclusive_scan(local, buf, &excl);
+  const int64_t total = block_exclusive_scan(local, warp_tot, &excl);
   for (int T = t0; T < t1; ++T) {
+    prefix_sm[T] = int32_t(excl);
+    tiles[size_t(T) * kTileInts + T_PAGES] = pages_sm[T];
     tiles[size_t(T) * kTileInts + T_PREFIX] = int32_t(excl);
-    excl += tile_cost(tiles[size_t(T) * kTileInts + T_PAGES]);
+    excl += tile_cost(pages_sm[T]);
   }
   __syncthreads();
 
-  // 3: worker start positions (end = next worker's start)
+  // 3: worker start positions (only min(W, total) workers get work)
+  const int64_t We = total < W ? total : W;
   for (int w = tid; w < W; w += kSchedThreads) {
-    int tile, page;
-    worker_start(tiles, num_tiles, total, w, W, &tile, &page);
-    int32_t* wm = workers + size_t(w) * kWorkerInts;
-    wm[W_TILE_BEGIN] = tile;
-    wm[W_PAGE_BEGIN] = page;
-    for (int k = W_FIRST_SPLIT; k < kWorkerInts; ++k) wm[k] = 0;
+    int tile = num_tiles, page = 0;
+    if (w < We) {
+      const int64_t x = total * w / We;
+      tile = last_le(prefix_sm, 1, num_tiles, x);
+      const int64_t pg = x - int64_t(prefix_sm[tile]) - kPieceOverhead;
+      page = pg > 0 ? int(pg) : 0;
+    }
+    wkey[w] = tp_key(tile, page);
   }
   __syncthreads();
   for (int w = tid; w < W; w += kSchedThreads) {
+    const int64_t k0 = wkey[w];
+    const int64_t k1 = w + 1 < W ? wkey[w + 1] : tp_key(num_tiles, 0);
     int32_t* wm = workers + size_t(w) * kWorkerInts;
-    if (w + 1 < W) {
-      wm[W_TILE_END] = workers[size_t(w + 1) * kWorkerInts + W_TILE_BEGIN];
-      wm[W_PAGE_END] = workers[size_t(w + 1) * kWorkerInts + W_PAGE_BEGIN];
-    } else {
-      wm[W_TILE_END] = num_tiles;
-      wm[W_PAGE_END] = 0;
-    }
-    if (wm[W_PAGE_BEGIN] > 0) {
-      int lo = first_worker_ge(workers, W, tp_key(wm[W_TILE_BEGIN], 1));
-      wm[W_FIRST_SPLIT] = w - lo + 1;
-    }
+    wm[W_TILE_BEGIN] = int32_t(k0 >> 32);
+    wm[W_PAGE_BEGIN] = int32_t(uint32_t(k0));
+    wm[W_TILE_END] = int32_t(k1 >> 32);
+    wm[W_PAGE_END] = int32_t(uint32_t(k1));
+    int first = 0;
+    if (uint32_t(k0) > 0) first = w - first_key_ge(wkey, W, tp_key(int32_t(k0 >> 32), 1)) + 1;
+    wm[W_FIRST_SPLIT] = first;
+    for (int k = W_FIRST_SPLIT + 1; k < kWorkerInts; ++k) wm[k] = 0;
   }
 
   // 4-5: pieces per tile and the base of their partial slots
   int64_t slots = 0;
   for (int T = t0; T < t1; ++T) {
-    int32_t* tm = tiles + size_t(T) * kTileInts;
     int n = 0;
-    if (tm[T_PAGES] > 0) {
-      int lo = first_worker_ge(workers, W, tp_key(T, 1));
-      int hi = first_worker_ge(workers, W, tp_key(T + 1, 0));
-      n = 1 + (hi - lo);
-    }
-    tm[T_SPLITS] = n;
+    if (pages_sm[T] > 0)
+      n = 1 + first_key_ge(wkey, W, tp_key(T + 1, 0)) - first_key_ge(wkey, W, tp_key(T, 1));
+    tiles[size_t(T) * kTileInts + T_SPLITS] = n;
     slots += n > 1 ? n : 0;
   }
   int64_t sexcl;
-  const int64_t slot_total = block_exclusive_scan(slots, buf, &sexcl);
+  const int64_t slot_total = block_exclusive_scan(slots, warp_tot, &sexcl);
   for (int T = t0; T < t1; ++T) {
-    int32_t* tm = tiles + size_t(T) * kTileInts;
-    tm[T_SLOT_BASE] = int32_t(sexcl);
-    sexcl += tm[T_SPLITS] > 1 ? tm[T_SPLITS] : 0;
+    const int n = tiles[size_t(T) * kTileInts + T_SPLITS];
+    tiles[size_t(T) * kTileInts + T_SLOT_BASE] = int32_t(sexcl);
+    sexcl += n > 1 ? n : 0;
   }
   if (tid == 0) {
     fill_header(hdr, s, W, num_tiles);
@@ -177,8 +212,9 @@ schedule_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t
 
 }  // namespace
 
-// Sequential host copy of schedule_kernel (identical results).
-void plan_schedule_host(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched) {
+// Sequential form of schedule_kernel (identical results): the host planner,
+// and the device fallback for oversized schedules.
+MLA_HD void plan_schedule_seq(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched) {
   const int num_tiles = s.batch * s.tiles_per_req;
   int32_t* hdr = sched;
   int32_t* workers = sched + kHeaderInts;
@@ -234,9 +270,32 @@ void plan_schedule_host(const int32_t* seqlens, const ShapeInfo& s, int W, int32
   hdr[H_STATUS] = flag;
 }
 
+void plan_schedule_host(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched) {
+  plan_schedule_seq(seqlens, s, W, sched);
+}
+
+namespace {
+// Schedules whose tables do not fit in shared memory: one thread runs the
+// sequential planner on the global copies (slow, but only for batches of
+// tens of thousands of tiles).
+__global__ void schedule_kernel_global(const int32_t* seqlens, ShapeInfo s, int W, int32_t* sched) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) plan_schedule_seq(seqlens, s, W, sched);
+}
+}  // namespace
+
 cudaError_t launch_schedule(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
                             cudaStream_t stream) {
-  schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seqlens, s, W, sched);
+  const size_t smem = sched_smem_bytes(s.batch * s.tiles_per_req, W);
+  if (smem <= kSchedSmemMax) {
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 int(kSchedSmemMax));
+      if (e != cudaSuccess) return e;
+    }
+    schedule_kernel<<<1, kSchedThreads, smem, stream>>>(seqlens, s, W, sched);
+  } else {
+    schedule_kernel_global<<<1, 32, 0, stream>>>(seqlens, s, W, sched);
+  }
   return cudaGetLastError();
 }
 
