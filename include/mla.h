@@ -158,6 +158,32 @@ int mla_get_device_status(const void* sched, void* workspace, void* stream, int*
 int mla_plan_schedule_host(const mla_shape_t* shape, const int32_t* seqlens, int num_sms,
                            void* sched, size_t sched_bytes);
 
+/* The pages have no counterpart to this call: it is the whole decode step
+ * (schedule, decode, combine) for callers that cannot allocate device
+ * memory -- a host program linking only this C ABI with no device allocator
+ * of its own, or a serving loop whose memory is entirely reserved up front --
+ * and so cannot pass the sched and workspace buffers that mla_get_schedule /
+ * mla_decode_fwd / mla_combine take.  It allocates nothing: its schedule and
+ * its device status word live in a static device array of 320 KiB inside
+ * the library (one per device), whose address is looked up with
+ * cudaGetSymbolAddress on the first call on each device; that first call
+ * must therefore not be made while `stream` is being captured.  To fit that
+ * array, work is assigned to the SM pairs in whole 128-row tiles (no tile is
+ * split, no fp32 partial result is kept), so a batch with one very long
+ * request balances worse than with mla_get_schedule.
+ *   Limit: batch * ceil(s_q * num_heads / 128) <= 16384 tiles; larger
+ *   shapes return MLA_ERR_WORKSPACE before anything is enqueued.
+ *   Arguments as for mla_decode_fwd; device_status: optional device int32
+ *   (4-byte aligned) that receives, in stream order, this call's status
+ *   word (0, or the bits behind MLA_ERR_TIMEOUT / MLA_ERR_DEVICE_CHECK);
+ *   NULL to skip.  The call zeroes the status word before its kernels run.
+ * Calls that overlap in time on one device (different streams, or threads
+ * without ordering) share the static array and race: serialise them. */
+int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, const void* kv_cache,
+                           const float* kv_scale, const int32_t* block_table,
+                           const int32_t* seqlens, float softmax_scale, void* out, float* lse,
+                           int32_t* device_status, void* stream);
+
 /* Human-readable name of an MLA_* code (static storage). */
 const char* mla_error_string(int code);
 

@@ -26,7 +26,7 @@ FP8_PAGE_BYTES = PAGE * D_V + PAGE * (D_QK - D_V) * 2
 
 EXPORTED = ("mla_schedule_bytes", "mla_workspace_bytes", "mla_get_schedule", "mla_decode_fwd",
             "mla_combine", "mla_decode_fwd_simt", "mla_get_device_status", "mla_plan_schedule_host",
-            "mla_error_string", "mla_version")
+            "mla_error_string", "mla_version", "mla_decode_fwd_noalloc")
 
 
 class MLAError(RuntimeError):
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.mla_get_device_status.restype = i32
         L.mla_plan_schedule_host.argtypes = [sp, vp, i32, vp, sz]
         L.mla_plan_schedule_host.restype = i32
+        L.mla_decode_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
+        L.mla_decode_fwd_noalloc.restype = i32
         L.mla_error_string.argtypes = [i32]
         L.mla_error_string.restype = ctypes.c_char_p
         L.mla_version.argtypes = []
@@ -144,6 +146,22 @@ def mla_plan_schedule_host(shape: mla_shape_t, seqlens: torch.Tensor, n_sms: int
     return out
 
 
+def _check_decode_tensors(shape, q, kv_cache, kv_scale, block_table, seqlens, out, lse):
+    b, s, h = shape.batch, shape.s_q, shape.num_heads
+    _need(q, "q", torch.bfloat16, (b, s, h, D_QK))
+    if shape.cache_dtype == MLA_CACHE_BF16:
+        _need(kv_cache, "kv_cache", torch.bfloat16, (shape.num_pages, PAGE, D_QK))
+        if kv_scale is not None:
+            raise ValueError("kv_scale is only used with the fp8 cache")
+    else:
+        _need(kv_cache, "kv_cache", torch.uint8, (shape.num_pages, FP8_PAGE_BYTES))
+        _need(kv_scale, "kv_scale", torch.float32, (shape.num_pages, PAGE))
+    _need(block_table, "block_table", torch.int32, (b, shape.max_pages_per_seq))
+    _need(seqlens, "seqlens", torch.int32, (b,))
+    _need(out, "out", torch.bfloat16, (b, s, h, D_V))
+    _need(lse, "lse", torch.float32, (b, s, h))
+
+
 def _decode_common(fn, where, shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched,
                    workspace, out, lse, stream):
     b, s, h = shape.batch, shape.s_q, shape.num_heads
@@ -177,6 +195,19 @@ def mla_decode_fwd_simt(shape, q, kv_cache, kv_scale, block_table, seqlens, soft
                         lse, stream=None):
     _decode_common(lib().mla_decode_fwd_simt, "mla_decode_fwd_simt", shape, q, kv_cache, kv_scale, block_table,
                    seqlens, softmax_scale, sched, workspace, out, lse, stream)
+
+
+def mla_decode_fwd_noalloc(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, out, lse,
+                           device_status: Optional[torch.Tensor] = None, stream=None):
+    """The whole decode step (schedule, decode, combine) with the library's
+    static scratch instead of caller buffers; see mla.h for its limits."""
+    _check_decode_tensors(shape, q, kv_cache, kv_scale, block_table, seqlens, out, lse)
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32)
+    rc = lib().mla_decode_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(kv_cache), _ptr(kv_scale),
+                                      _ptr(block_table), _ptr(seqlens), float(softmax_scale), _ptr(out), _ptr(lse),
+                                      _ptr(device_status), _stream(stream))
+    _check(rc, "mla_decode_fwd_noalloc")
 
 
 def mla_combine(shape, sched, workspace, out, lse, stream=None):

@@ -283,6 +283,99 @@ __global__ void schedule_kernel_global(const int32_t* seqlens, ShapeInfo s, int 
 }
 }  // namespace
 
+namespace {
+// Whole-tile variant of schedule_kernel, for the no-allocation entry point:
+// worker w starts at the first tile whose cost prefix is >= total*w/W_eff,
+// so worker boundaries fall on tile starts, no tile is split and no partial
+// slot is ever used.  Same schedule format (every split count is 1, or 0 for
+// a tile with no visible key), so the decode and combine kernels run on it
+// unchanged.  The balance is coarser than schedule_kernel's: a worker's share
+// is rounded to whole tiles.  Invalid lengths are flagged in the schedule
+// header and in *status.
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_whole_tiles_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t* __restrict__ sched,
+                            int32_t* __restrict__ status) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ int64_t warp_tot[kSchedWarps];
+  __shared__ int32_t flag_sh;
+  const int tid = threadIdx.x;
+  const int num_tiles = s.batch * s.tiles_per_req;
+  int32_t* pages_sm = reinterpret_cast<int32_t*>(smem);
+  int32_t* prefix_sm = pages_sm + num_tiles;
+  int32_t* hdr = sched;
+  int32_t* workers = sched + kHeaderInts;
+  int32_t* tiles = workers + size_t(W) * kWorkerInts;
+  if (tid == 0) flag_sh = 0;
+  __syncthreads();
+
+  const int chunk = (num_tiles + kSchedThreads - 1) / kSchedThreads;
+  const int t0 = min(num_tiles, tid * chunk), t1 = min(num_tiles, t0 + chunk);
+  int32_t flag = 0;
+  int64_t local = 0;
+  for (int T = t0; T < t1; ++T) {
+    const int r = T / s.tiles_per_req, qt = T % s.tiles_per_req;
+    const int pages = tile_pages(s, clamp_seqlen(seqlens[r], s.max_pages, &flag), qt);
+    pages_sm[T] = pages;
+    local += tile_cost(pages);
+  }
+  if (flag) atomicOr(&flag_sh, flag);
+  int64_t excl;
+  const int64_t total = block_exclusive_scan(local, warp_tot, &excl);
+  for (int T = t0; T < t1; ++T) {
+    prefix_sm[T] = int32_t(excl);
+    int32_t* tm = tiles + size_t(T) * kTileInts;
+    tm[T_PAGES] = pages_sm[T];
+    tm[T_PREFIX] = int32_t(excl);
+    tm[T_SPLITS] = pages_sm[T] > 0 ? 1 : 0;
+    tm[T_SLOT_BASE] = 0;
+    excl += tile_cost(pages_sm[T]);
+  }
+  __syncthreads();
+
+  const int64_t We = total < W ? total : W;
+  for (int w = tid; w < W; w += kSchedThreads) {
+    int32_t* wm = workers + size_t(w) * kWorkerInts;
+    int tb = num_tiles, te = num_tiles;
+    if (w < We) {
+      // first tile with prefix >= x (prefix non-decreasing)
+      const int64_t x = total * w / We, x1 = total * (w + 1) / We;
+      tb = last_le(prefix_sm, 1, num_tiles, x - 1) + 1;
+      te = w + 1 < We ? last_le(prefix_sm, 1, num_tiles, x1 - 1) + 1 : num_tiles;
+    }
+    wm[W_TILE_BEGIN] = tb;
+    wm[W_PAGE_BEGIN] = 0;
+    wm[W_TILE_END] = te;
+    wm[W_PAGE_END] = 0;
+    for (int k = W_FIRST_SPLIT; k < kWorkerInts; ++k) wm[k] = 0;
+  }
+  if (tid == 0) {
+    fill_header(hdr, s, W, num_tiles);
+    hdr[H_TOTAL_COST] = int32_t(total);
+    hdr[H_MAX_SLOTS] = 0;
+    hdr[H_STATUS] = flag_sh;
+    if (flag_sh) atomicOr(status, flag_sh);
+  }
+}
+}  // namespace
+
+// Shared-memory bytes the whole-tile scheduler needs (0 when it cannot run).
+size_t schedule_whole_tiles_smem(int num_tiles) {
+  const size_t b = size_t(num_tiles) * 8;
+  return b <= kSchedSmemMax ? b : 0;
+}
+
+cudaError_t launch_schedule_whole_tiles(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
+                                        int32_t* status, cudaStream_t stream) {
+  const size_t smem = size_t(s.batch) * s.tiles_per_req * 8;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(schedule_whole_tiles_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSchedSmemMax));
+    if (e != cudaSuccess) return e;
+  }
+  schedule_whole_tiles_kernel<<<1, kSchedThreads, smem, stream>>>(seqlens, s, W, sched, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_schedule(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
                             cudaStream_t stream) {
   const size_t smem = sched_smem_bytes(s.batch * s.tiles_per_req, W);

@@ -220,3 +220,20 @@ def test_schedule_clamps_bad_lengths():
     sc = parse_schedule(buf, shape)
     assert sc["hdr"][6] != 0                       # status flags the clamp
     assert list(sc["tiles"][:, 0]) == [0, 2, 1]
+
+
+def test_noalloc_rejects_shapes_beyond_its_static_scratch():
+    """mla_decode_fwd_noalloc checks its size limit (16384 tiles) on the host
+    before any CUDA call; the pointers are never touched."""
+    L = mla.lib()
+    fake = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+    for batch, s_q, heads in ((16385, 1, 128), (1, 16385, 128), (8193, 2, 128)):
+        shape = mla.make_shape(batch, s_q, heads, 4, 16)
+        rc = L.mla_decode_fwd_noalloc(ctypes.byref(shape), fake, fake, None, fake, fake, 0.1, fake, fake, None,
+                                      None)
+        assert rc == -3, (batch, s_q, heads, rc)
+    shape = mla.make_shape(2, 1, 128, 4, 16)
+    shape.d_qk = 512
+    assert L.mla_decode_fwd_noalloc(ctypes.byref(shape), fake, fake, None, fake, fake, 0.1, fake, fake, None,
+                                    None) == -2
+    assert L.mla_decode_fwd_noalloc(None, fake, fake, None, fake, fake, 0.1, fake, fake, None, None) == -1
