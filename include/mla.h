@@ -122,11 +122,13 @@ int mla_get_schedule(const mla_shape_t* shape, const int32_t* seqlens, int num_s
  *                aligned; the caller must not touch it between this call and
  *                mla_combine.
  *   out        : bf16 [batch, s_q, num_heads, 512], the latent output rows.
- *                BF16 cache: the tensor-core kernel (tcgen05, 2-SM clusters),
- *                which rounds P to fp16 and converts V to fp16 on chip, so
- *                cache values must lie within fp16 range (|v| < 65504).
- *                FP8 cache: runs the SIMT kernel of mla_decode_fwd_simt (a
- *                tensor-core FP8 kernel is not built yet).
+ *                The tensor-core kernel (tcgen05, 2-SM clusters) rounds P to
+ *                fp16 and converts V to fp16 on chip, so value rows must lie
+ *                within fp16 range (|v| < 65504; FP8: |e4m3 * scale|).  FP8
+ *                cache: the latent scores use e4m3 -> fp16 (exact) against an
+ *                fp16 copy of the query's latent part, so those query values
+ *                must lie within fp16 range too; a value outside it is flagged
+ *                (MLA_ERR_DEVICE_CHECK from mla_get_device_status).
  *   lse        : fp32 [batch, s_q, num_heads], natural-log log-sum-exp of the
  *                scaled scores (-inf for a row that sees no key).
  * Tiles cut into several pieces are finished by mla_combine; tiles in one
@@ -143,9 +145,9 @@ int mla_decode_fwd(const mla_shape_t* shape, const void* q, const void* kv_cache
 int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace,
                 size_t workspace_bytes, void* out, float* lse, void* stream);
 
-/* The same decode computed by a plain SIMT kernel (fp32 FMA, no tensor
- * cores) over the same schedule and workspace.  The tests use it as a second
- * implementation; mla_decode_fwd runs it for the FP8 cache only. */
+/* Debug path, used by the tests only: the same decode computed by a plain
+ * SIMT kernel (fp32 FMA, no tensor cores) over the same schedule and
+ * workspace.  Never chosen by mla_decode_fwd. */
 int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_cache,
                         const float* kv_scale, const int32_t* block_table,
                         const int32_t* seqlens, float softmax_scale, const void* sched,

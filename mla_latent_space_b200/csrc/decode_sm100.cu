@@ -54,7 +54,9 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring
+constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring (bf16 cache)
+constexpr int NZ8 = 6;  // the same ring for the FP8 cache (e4m3 and RoPE stages)
+constexpr int NC = 4;   // FP8 cache: 16 KB stages of fp16 cache rows converted from e4m3
 constexpr int NX = 1;   // P block stages (output CTA)
 constexpr int NV = 3;   // V page stages (output CTA): its own TMA ring
 // Per-block PV completion barriers for the correction warpgroup.  It may lag
@@ -80,10 +82,15 @@ constexpr float kLazyMax = 8.0f;                      // log2 units
 constexpr int kConvThreads = 256;                     // output-CTA warps 8..15
 constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
 constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of the softmax warps
+constexpr uint32_t kConvBar = 2;                      // named barrier of a CTA's converter warps
+constexpr int kConvThreadsS = 128;                    // FP8 cache: score-CTA converters, warps 12..15
+constexpr uint32_t kFp8PageBytes = 64 * 512 + 64 * 64 * 2;   // 64x512 e4m3, then 64x64 bf16 RoPE
+constexpr uint32_t kTmemSLat = 256;                   // FP8 cache: latent-part scores, columns 256..383
 
 struct Bars {
-  // score CTA
+  // score CTA (FP8 cache: also the converted ring and the query RoPE buffer)
   uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
+  uint64_t c_full[NC], c_empty[NC], qpe_full, qpe_empty;
   // output CTA
   uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], pv_blk[NB], o_free;
   // both
@@ -94,11 +101,21 @@ struct Bars {
 };
 
 constexpr uint32_t kOffData = 1024;
-// score CTA
-constexpr uint32_t kOffZ = kOffData;
-constexpr uint32_t kOffStage = kOffZ + NZ * kZStage;          // P staging (local, one block)
-constexpr uint32_t kOffXchg = kOffStage + kPStage;            // row max / sum exchange
-constexpr uint32_t kSmemS = kOffXchg + 4 * 128 * 4;
+// score CTA.  BF16 cache: ring | P staging | exchange.  FP8 cache: ring |
+// converted ring | query RoPE columns (128 rows x 64, one 16 KB stage) |
+// P staging | exchange | per-token scales of the block's two pages.
+template <bool kFp8>
+struct LayS {
+  static constexpr int nz = kFp8 ? NZ8 : NZ;
+  static constexpr uint32_t z = kOffData;
+  static constexpr uint32_t c = z + nz * kZStage;
+  static constexpr uint32_t qpe = c + (kFp8 ? NC * kZStage : 0u);
+  static constexpr uint32_t stage = qpe + (kFp8 ? kZStage : 0u);
+  static constexpr uint32_t xchg = stage + kPStage;               // row max / sum exchange
+  static constexpr uint32_t scales = xchg + 4 * 128 * 4;           // FP8: 2 x 64 fp32
+  static constexpr uint32_t end = scales + (kFp8 ? 2 * 64 * 4 : 0u);
+};
+constexpr uint32_t kSmemS = LayS<false>::end > LayS<true>::end ? LayS<false>::end : LayS<true>::end;
 // output CTA
 constexpr uint32_t kOffV = kOffData;
 constexpr uint32_t kOffP = kOffV + NV * kVStage;              // P + meta block stages
@@ -107,6 +124,7 @@ constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // 
 static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kPStage % 1024 == 0 && kZStage % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(LayS<true>::c % 1024 == 0 && LayS<true>::qpe % 1024 == 0 && LayS<true>::stage % 1024 == 0, "align");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
 //   QK: A = Q bf16 (TMEM), B = cache rows bf16 K-major, N = 128
@@ -114,6 +132,8 @@ static_assert(kPStage % 1024 == 0 && kZStage % 1024 == 0, "swizzle atoms need 10
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((256u >> 3) << 17) |
                               ((128u >> 4) << 24);
+//   FP8 cache, latent part: A = Q fp16 (TMEM), B = converted rows fp16 K-major, N = 128
+constexpr uint32_t kIdescQKh = (1u << 4) | (0u << 7) | (0u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 // Shared-memory matrix descriptor, 128-byte swizzle.  lbo / sbo in bytes.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -124,6 +144,7 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
 struct Params {
   const uint16_t* q;
   const uint8_t* kv;
+  const float* kv_scale;   // FP8 cache: per-token scales [pages][64]
   const int32_t* block_table;
   const int32_t* seqlens;
   const void* sched;
@@ -139,17 +160,21 @@ struct Params {
 
 // Optional device event trace.  Built only with -DMLA_TRACE: one thread per
 // role of cluster 0 records (event << 24 | index, clock64, 0) into
-// trace[role][2048][3]; roles 6 and 7 hold one (0, clock64, %globaltimer)
-// pair per CTA taken right after the start-up cluster barrier, to line the
-// two SMs' clocks up.  Only the SM clock is read per event (the global timer
+// trace[role][2048][3]; the last entry of roles 6 and 7 holds one
+// (0, clock64, %globaltimer) pair per CTA taken right after the start-up
+// cluster barrier, to line the two SMs' clocks up (role 6 also records the
+// score CTA's FP8 converters).  Only the SM clock is read per event (the global timer
 // is far slower to read and would distort the timeline).  In normal builds
 // the hooks compile to nothing.
 #ifdef MLA_TRACE
+#ifndef MLA_TRACE_CLUSTER
+#define MLA_TRACE_CLUSTER 0
+#endif
 #define MLA_TR(role, ev, j)                                                               \
   do {                                                                                    \
-    if (p.trace && cluster_id_x() == 0) {                                                 \
+    if (p.trace && cluster_id_x() == MLA_TRACE_CLUSTER) {                                                 \
       const unsigned k_ = bars->trc[role]++;                                              \
-      if (k_ < 2048) {                                                                    \
+      if (k_ < 2047) {                                                                    \
         unsigned long long* e_ = p.trace + (size_t(role) * 2048 + k_) * 3;                \
         e_[0] = (unsigned long long)(((ev) << 24) | (unsigned(j) & 0xFFFFFF));            \
         e_[1] = clock64();                                                                \
@@ -158,8 +183,8 @@ struct Params {
   } while (0)
 #define MLA_TR_SYNC(role)                                                                 \
   do {                                                                                    \
-    if (p.trace && cluster_id_x() == 0) {                                                 \
-      unsigned long long* e_ = p.trace + size_t(role) * 2048 * 3;                         \
+    if (p.trace && cluster_id_x() == MLA_TRACE_CLUSTER) {                                                 \
+      unsigned long long* e_ = p.trace + (size_t(role) * 2048 + 2047) * 3;                \
       e_[1] = clock64();                                                                  \
       e_[2] = globaltimer();                                                              \
     }                                                                                     \
@@ -250,6 +275,28 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Two e4m3 bytes (low byte first) -> two fp16 (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+  return uint32_t(h.x) | (uint32_t(h.y) << 16);
+}
+
+// The same, times a per-token scale (fp16 product, one rounding).
+__device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two, __half2 scale) {
+  const uint32_t w = e4m3x2_to_f16x2(two);
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&w), scale);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// bf16 pair -> fp16 pair (exact inside fp16's range); *big records a value
+// outside it (or NaN).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_checked(uint32_t w, bool* big) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+  *big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -283,9 +330,13 @@ __device__ __forceinline__ int clamp_len(int t, const SchedView& sv) {
   return max(0, min(t, sv.max_pages * MLA_PAGE_SIZE));
 }
 
+// kFp8: the cache pages hold e4m3 latent values with per-token scales and a
+// bf16 RoPE part (pool_map covers the e4m3 bytes, rope_map the RoPE values);
+// otherwise pool_map covers bf16 rows and rope_map is not used.
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_constant__ CUtensorMap q_map,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap rope_map, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -297,7 +348,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   const uint32_t rank = cluster_ctarank();
 
   if (tid == 0) {
-    for (int s = 0; s < NZ; ++s) { mbar_init(bar(bars->z_full[s]), 1); mbar_init(bar(bars->z_empty[s]), 1); }
+    // FP8 cache: a ring stage is refilled once the softmax, the issuer and
+    // the converters have each released it (see the issuer)
+    for (int s = 0; s < NZ; ++s) {
+      mbar_init(bar(bars->z_full[s]), 1);
+      mbar_init(bar(bars->z_empty[s]), kFp8 ? 3 : 1);
+    }
     mbar_init(bar(bars->s_full), 1);
     mbar_init(bar(bars->s_empty), kSmThreads);
     mbar_init(bar(bars->q_ready), kSmThreads);
@@ -312,6 +368,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       mbar_init(bar(bars->pv_done[s]), 1);
     }
     for (int s = 0; s < NB; ++s) mbar_init(bar(bars->pv_blk[s]), 1);
+    for (int s = 0; s < NC; ++s) {
+      mbar_init(bar(bars->c_full[s]), kConvThreadsS);
+      mbar_init(bar(bars->c_empty[s]), 1);
+    }
+    mbar_init(bar(bars->qpe_full), 1);
+    mbar_init(bar(bars->qpe_empty), 1);
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
@@ -324,6 +386,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&pool_map);
     if (rank == 0) tma_prefetch_desc(&q_map);
+    if (kFp8 && rank == 0) tma_prefetch_desc(&rope_map);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), 512);
@@ -346,19 +409,25 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 
   if (rank == 0) {
     // ======================= score CTA =======================
+    using L = LayS<kFp8>;
+    constexpr int nz = L::nz;
     if (warp == 0) {
-      if (lane == 0) {  // ---- TMA producer: 9 query stages per piece, then 9 per 2-page block
-        uint32_t zc = 0;
+      // ---- TMA producer.  BF16 cache: 9 query stages per piece, then 9 per
+      // 2-page block.  FP8 cache: 8 query stages (latent columns) plus the
+      // query RoPE columns into their own buffer per piece, then per block one
+      // RoPE stage (bf16) and 4 e4m3 stages of 128 latent columns.
+      if (lane == 0) {
+        uint32_t zc = 0, pieces = 0;
         auto page_of = [&](int r, int j) {
           int page = p.block_table[size_t(r) * sv.max_pages + j];
           return (page < 0 || page >= p.num_pages) ? -1 : page;
         };
         auto stage = [&](uint32_t tx, uint32_t* dst) -> bool {
-          const uint32_t s = zc % NZ, ph = (zc / NZ) & 1u;
+          const uint32_t s = zc % nz, ph = (zc / nz) & 1u;
           if (!swait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
           MLA_TR(0, 1, zc);
           mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
-          *dst = sbase + kOffZ + s * kZStage;
+          *dst = sbase + L::z + s * kZStage;
           return true;
         };
         each_piece(sv, [&](const Piece& pc) {
@@ -366,81 +435,221 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const int row0 = r * rows_total + qt * MLA_TILE_ROWS;
           prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK,
                            uint32_t(min(MLA_TILE_ROWS, p.q_rows - row0)) * MLA_D_QK * 2);
-          for (int j = pc.p0; j < min(pc.p1, pc.p0 + kPrefetchPages); ++j) {
-            const int pg = page_of(r, j);
-            if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
-          }
-          for (int c = 0; c < 9; ++c, ++zc) {
+          for (int c = 0; c < (kFp8 ? 8 : 9); ++c, ++zc) {
             uint32_t dst;
             if (!stage(kZStage, &dst)) return false;
-            const uint32_t fb = bar(bars->z_full[zc % NZ]);
+            const uint32_t fb = bar(bars->z_full[zc % nz]);
             tma_load_2d(dst, &q_map, 64 * c, row0, fb);
             tma_load_2d(dst + kBox, &q_map, 64 * c, row0 + 64, fb);
           }
+          if constexpr (kFp8) {
+            // the RoPE MMAs of the previous piece must be done with the buffer
+            if (!swait(ctl, bar(bars->qpe_empty), (pieces & 1u) ^ 1u)) return false;
+            const uint32_t fb = bar(bars->qpe_full);
+            mbar_arrive_expect_tx(fb, kZStage);
+            tma_load_2d(sbase + L::qpe, &q_map, MLA_D_V, row0, fb);
+            tma_load_2d(sbase + L::qpe + kBox, &q_map, MLA_D_V, row0 + 64, fb);
+          }
+          ++pieces;
           for (int j = pc.p0; j < pc.p1; j += 2) {
             const bool two = j + 1 < pc.p1;
-            for (int u = 0; u < 2; ++u)
-              if (kPrefetchPages > 0 && j + u + kPrefetchPages < pc.p1) {
-                const int pg = page_of(r, j + u + kPrefetchPages);
-                if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
-              }
+            if constexpr (!kFp8) {
+              for (int u = 0; u < 2; ++u)
+                if (kPrefetchPages > 0 && j + u + kPrefetchPages < pc.p1) {
+                  const int pg = page_of(r, j + u + kPrefetchPages);
+                  if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
+                }
+            }
             int pa = page_of(r, j), pb = two ? page_of(r, j + 1) : 0;
             if (pa < 0 || pb < 0) flag_status(p.ws, kStatusBadPage);
             pa = max(pa, 0);     // any valid page; the consumers mask every token of it
             pb = max(pb, 0);
-            for (int c = 0; c < 9; ++c, ++zc) {
+            if constexpr (kFp8) {
               uint32_t dst;
               if (!stage(two ? kZStage : kBox, &dst)) return false;
-              const uint32_t fb = bar(bars->z_full[zc % NZ]);
-              tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
-              if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
+              uint32_t fb = bar(bars->z_full[zc % nz]);
+              tma_load_3d(dst, &rope_map, 0, 0, pa, fb);
+              if (two) tma_load_3d(dst + kBox, &rope_map, 0, 0, pb, fb);
+              ++zc;
+              for (int c = 0; c < 4; ++c, ++zc) {
+                if (!stage(two ? kZStage : kBox, &dst)) return false;
+                fb = bar(bars->z_full[zc % nz]);
+                tma_load_3d(dst, &pool_map, 128 * c, 0, pa, fb);
+                if (two) tma_load_3d(dst + kBox, &pool_map, 128 * c, 0, pb, fb);
+              }
+            } else {
+              for (int c = 0; c < 9; ++c, ++zc) {
+                uint32_t dst;
+                if (!stage(two ? kZStage : kBox, &dst)) return false;
+                const uint32_t fb = bar(bars->z_full[zc % nz]);
+                tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
+                if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
+              }
             }
           }
           return true;
         });
         // copies still in flight must land before the CTA can leave
-        const uint32_t n = zc < NZ ? zc : NZ;
+        const uint32_t n = zc < uint32_t(nz) ? zc : uint32_t(nz);
         for (uint32_t k = 1; k <= n; ++k) {
           const uint32_t idx = zc - k;
-          drain_wait(bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u);
+          drain_wait(bar(bars->z_full[idx % nz]), (idx / nz) & 1u);
         }
+        if (kFp8 && pieces > 0) drain_wait(bar(bars->qpe_full), (pieces - 1) & 1u);
       }
     } else if (warp == 1) {
-      if (lane == 0) {  // ---- QK^T issuer: per block 9 stages x 4 MMAs (N = 128)
-        const uint64_t zdesc0 = sdesc(sbase + kOffZ, 16, 1024);
-        uint32_t zc = 0, bc = 0, pieces = 0;
+      // ---- QK^T issuer: per block 36 MMAs M128 N128 K16.  BF16 cache: 9
+      // stages x 4, A = Q (TMEM), into S.  FP8 cache: the RoPE stage x 4 with
+      // A = the query RoPE columns (shared memory) into S_rope, then 8
+      // converted fp16 stages x 4 with A = the fp16 query (TMEM) into S_lat.
+      if (lane == 0) {
+        const uint64_t zdesc0 = sdesc(sbase + L::z, 16, 1024);
+        const uint64_t cdesc0 = sdesc(sbase + L::c, 16, 1024);
+        const uint64_t qdesc = sdesc(sbase + L::qpe, 16, 1024);
+        uint32_t zc = 0, cc = 0, bc = 0, pieces = 0;
         each_piece(sv, [&](const Piece& pc) {
+          // FP8 cache: the ring is shorter than the query, so its stages are
+          // released one by one.  This thread and one converter thread walk
+          // every stage of the ring in order (a parity wait is only sound when
+          // the stage's previous use has completed), and a stage is refilled
+          // after three releases: softmax, issuer, converter.  For the RoPE
+          // and e4m3 stages, which the softmax never sees, the issuer releases
+          // twice.
+          constexpr int nq = kFp8 ? 8 : 9;
+          if constexpr (kFp8) {
+            for (int u = 0; u < nq; ++u, ++zc) {
+              if (!swait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
+              mbar_arrive(bar(bars->z_empty[zc % nz]));
+            }
+          }
           if (!swait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
+          if (kFp8 && !swait(ctl, bar(bars->qpe_full), pieces & 1u)) return false;
           MLA_TR(1, 0, bc);
           ++pieces;
-          // the query rows are in TMEM: release their nine stages
-          for (int u = 0; u < 9; ++u) mbar_arrive(bar(bars->z_empty[(zc + u) % NZ]));
-          zc += 9;
+          // the query rows are in TMEM: release their stages
+          if constexpr (!kFp8) {
+            for (int u = 0; u < nq; ++u) mbar_arrive(bar(bars->z_empty[(zc + u) % nz]));
+            zc += nq;
+          }
           tc_fence_after();
           for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
             if (!swait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
             MLA_TR(1, 2, bc);
             tc_fence_after();
-            for (int c = 0; c < 9; ++c, ++zc) {
-              const uint32_t zs = zc % NZ;
-              if (!swait(ctl, bar(bars->z_full[zs]), (zc / NZ) & 1u)) return false;
-              MLA_TR(1, 10 + c, bc);
-              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
-              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
-              mma_ts(d, ad, bd, kIdescQK, c != 0);
-              mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
-              mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
-              mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
-              mma_commit(bar(bars->z_empty[zs]));
+            if constexpr (kFp8) {
+              {
+                const uint32_t zs = zc % nz;
+                if (!swait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
+                MLA_TR(1, 20, zc);
+                const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+                const uint32_t d = tmem + kTmemS;
+                mma_ss(d, qdesc, bd, kIdescQK, 0u);
+                mma_ss(d, qdesc + 2u, bd + 2u, kIdescQK, 1u);
+                mma_ss(d, qdesc + 4u, bd + 4u, kIdescQK, 1u);
+                mma_ss(d, qdesc + 6u, bd + 6u, kIdescQK, 1u);
+                mma_commit(bar(bars->z_empty[zs]));    // the issuer's release, when the MMAs are done
+                mbar_arrive(bar(bars->z_empty[zs]));   // the softmax's
+                ++zc;
+              }
+              for (int c = 0; c < 8; ++c, ++cc) {
+                if ((c & 1) == 0) {   // e4m3 stage c/2: observed in order, released for issuer and softmax
+                  if (!swait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
+                  mbar_arrive_cnt(bar(bars->z_empty[zc % nz]), 2u);
+                  ++zc;
+                }
+                const uint32_t cs = cc % NC;
+                if (!swait(ctl, bar(bars->c_full[cs]), (cc / NC) & 1u)) return false;
+                MLA_TR(1, 21, cc);
+                const uint64_t bd = cdesc0 + uint64_t(cs * (kZStage >> 4));
+                const uint32_t ad = tmem + 32u * c, d = tmem + kTmemSLat;
+                mma_ts(d, ad, bd, kIdescQKh, c != 0);
+                mma_ts(d, ad + 8u, bd + 2u, kIdescQKh, 1u);
+                mma_ts(d, ad + 16u, bd + 4u, kIdescQKh, 1u);
+                mma_ts(d, ad + 24u, bd + 6u, kIdescQKh, 1u);
+                mma_commit(bar(bars->c_empty[cs]));
+              }
+            } else {
+              for (int c = 0; c < 9; ++c, ++zc) {
+                const uint32_t zs = zc % nz;
+                if (!swait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
+                MLA_TR(1, 10 + c, bc);
+                const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+                const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
+                mma_ts(d, ad, bd, kIdescQK, c != 0);
+                mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
+                mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
+                mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
+                mma_commit(bar(bars->z_empty[zs]));
+              }
             }
             mma_commit(bar(bars->s_full));
             MLA_TR(1, 3, bc);
           }
+          if (kFp8) mma_commit(bar(bars->qpe_empty));   // the piece's RoPE MMAs are done with the buffer
           return true;
         });
         mma_commit(bar(bars->mma_done));
         drain_wait(bar(bars->mma_done), 0);
       }
+    } else if (kFp8 && warp >= 12) {
+      // ---- FP8 cache: converters.  Each e4m3 stage (128 latent columns of
+      // the block's two pages) becomes two fp16 stages of 64 columns in the
+      // K-major 128-byte-swizzled layout of the bf16 path.  e4m3 -> fp16 is
+      // exact.  Thread t owns token row t & 63 of page t >> 6.
+      const int t = tid - 384, pg = t >> 6, rr = t & 63;
+      const uint32_t sw = uint32_t(rr & 7);
+      uint32_t zc = 0, cc = 0;
+      // Thread 0 also walks the query and RoPE stages in order and releases
+      // them (the converters' share of their three releases).
+      bool ok = true;
+      auto observe = [&](uint32_t n) {
+        for (uint32_t u = 0; u < n; ++u, ++zc)
+          if (t == 0 && ok) {
+            ok = bwait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u);
+            if (ok) mbar_arrive(bar(bars->z_empty[zc % nz]));
+          }
+      };
+      each_piece(sv, [&](const Piece& pc) {
+        observe(8);                                // the query stages
+        for (int j = pc.p0; j < pc.p1; j += 2) {
+          observe(1);                              // the RoPE stage
+          for (int c = 0; c < 4; ++c, ++zc, cc += 2) {
+            const uint32_t zs = zc % nz, c0 = cc % NC, c1 = (cc + 1) % NC;
+            if (t == 0 && ok)
+              ok = bwait(ctl, bar(bars->c_empty[c0]), ((cc / NC) & 1u) ^ 1u) &&
+                   bwait(ctl, bar(bars->c_empty[c1]), (((cc + 1) / NC) & 1u) ^ 1u) &&
+                   bwait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u);
+            if (!named_bar_and(kConvBar, kConvThreadsS, ok)) return false;
+            if (t == 0) MLA_TR(6, 1, zc);
+            const uint32_t src = sbase + L::z + zs * kZStage + uint32_t(pg) * kBox + uint32_t(rr) * 128;
+            uint4 in[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) in[k] = ld_shared_v4(src + ((uint32_t(k) ^ sw) << 4));
+            // every converter has read the stage: the producer may refill it
+            named_bar_sync(kConvBar, kConvThreadsS);
+            if (t == 0) mbar_arrive(bar(bars->z_empty[zs]));
+            const uint32_t row = uint32_t(pg) * kBox + uint32_t(rr) * 128;
+            const uint32_t d0 = sbase + L::c + c0 * kZStage + row, d1 = sbase + L::c + c1 * kZStage + row;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              // 16 e4m3 values (latent columns 16k..16k+15 of the box) -> fp16
+              // chunks 2(k&3), 2(k&3)+1 of converted stage k >> 2
+              const uint32_t dst = (k < 4 ? d0 : d1);
+              const uint32_t ch = uint32_t(2 * (k & 3));
+              st_shared_v4(dst + ((ch ^ sw) << 4), e4m3x2_to_f16x2(in[k].x & 0xFFFFu), e4m3x2_to_f16x2(in[k].x >> 16),
+                           e4m3x2_to_f16x2(in[k].y & 0xFFFFu), e4m3x2_to_f16x2(in[k].y >> 16));
+              st_shared_v4(dst + (((ch + 1u) ^ sw) << 4), e4m3x2_to_f16x2(in[k].z & 0xFFFFu),
+                           e4m3x2_to_f16x2(in[k].z >> 16), e4m3x2_to_f16x2(in[k].w & 0xFFFFu),
+                           e4m3x2_to_f16x2(in[k].w >> 16));
+            }
+            fence_proxy_async_cta();   // the stages feed the tensor core
+            mbar_arrive(bar(bars->c_full[c0]));
+            mbar_arrive(bar(bars->c_full[c1]));
+            if (t == 0) MLA_TR(6, 2, zc);
+          }
+        }
+        return true;
+      });
     } else if (warp >= 4 && warp < 12) {
       // ---- softmax: two warpgroups; thread (h, i) owns row i of the tile
       // (TMEM lane i) for page h of each 2-page block
@@ -448,8 +657,9 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
       const uint32_t o_p = mapa(sbase + kOffP, 1);
       const uint32_t o_pfull = mapa(bar(bars->p_full[0]), 1);
-      const uint32_t stg = sbase + kOffStage;
-      const uint32_t xmax = sbase + kOffXchg, xsum = xmax + 2 * 128 * 4;
+      const uint32_t stg = sbase + L::stage;
+      const uint32_t xmax = sbase + L::xchg, xsum = xmax + 2 * 128 * 4;
+      const uint32_t scl = sbase + L::scales + uint32_t(h) * 256;   // FP8: this page's 64 scales
       uint32_t zc = 0, bc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
@@ -458,18 +668,25 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
         if (g == 0) MLA_TR(2, 9, bc);
-        // query row i -> TMEM lane i, columns [0, 288) (bf16 pairs).  Box c
-        // of the query is stage zc + c (rows 0-63, then 64-127 at +8 KB).
-        // Group 0 moves boxes 0-4, group 1 boxes 5-8.  Every QK MMA of the
-        // previous piece has completed: its last S was read.
+        // query row i -> TMEM lane i.  Box c of the query is stage zc + c
+        // (rows 0-63, then 64-127 at +8 KB).  BF16 cache: boxes 0-8 as bf16
+        // pairs in columns [0, 288), group 0 moves boxes 0-4, group 1 boxes
+        // 5-8.  FP8 cache: the latent boxes 0-7 as fp16 pairs in columns
+        // [0, 256) (the RoPE box stays in shared memory), 0-3 / 4-7.  Every QK
+        // MMA of the previous piece has completed: its last S was read.
         {
+          constexpr int nq = kFp8 ? 8 : 9, nq0 = kFp8 ? 4 : 5;
           const uint32_t roff = uint32_t(i >> 6) * kBox + uint32_t(i & 63) * 128;
+          bool big = false;
 #pragma unroll 1
-          for (int c = 0; c < 9; ++c) {
+          for (int c = 0; c < nq; ++c) {
             const uint32_t idx = zc + c;
-            if (!gwait(ctl, bar(bars->z_full[idx % NZ]), (idx / NZ) & 1u, g == 0)) return false;
-            if ((c < 5) == (h == 0)) {
-              const uint32_t st = sbase + kOffZ + (idx % NZ) * kZStage + roff;
+            if (!gwait(ctl, bar(bars->z_full[idx % nz]), (idx / nz) & 1u, g == 0)) return false;
+            // FP8 cache: every thread has passed the barrier, so the previous
+            // query stage has been read: the producer may refill it
+            if (kFp8 && c > 0 && g == 0) mbar_arrive(bar(bars->z_empty[(idx - 1) % nz]));
+            if ((c < nq0) == (h == 0)) {
+              const uint32_t st = sbase + L::z + (idx % nz) * kZStage + roff;
               uint32_t v[32];
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
@@ -479,10 +696,19 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                 v[4 * k + 2] = x.z;
                 v[4 * k + 3] = x.w;
               }
+              if constexpr (kFp8) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) v[k] = bf16x2_to_f16x2_checked(v[k], &big);
+              }
               tmem_st32(tmem + lane_off + 32u * c, v);
             }
           }
-          zc += 9 + 9 * ((pc.p1 - pc.p0 + 1) / 2);
+          if (kFp8 && big) flag_status(p.ws, kStatusBadInput);
+          if constexpr (kFp8) {
+            named_bar_sync(kSoftmaxBar, kSmThreads);
+            if (g == 0) mbar_arrive(bar(bars->z_empty[(zc + nq - 1) % nz]));
+          }
+          zc += nq + (kFp8 ? 5 : 9) * ((pc.p1 - pc.p0 + 1) / 2);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
@@ -490,28 +716,66 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
         float m = -INFINITY, l = 0.f;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          const int jp = j + h;                      // this thread's page
+          int nv = 0, page = -1;                     // its visible tokens here
+          if (jp < pc.p1) {
+            page = p.block_table[size_t(r) * sv.max_pages + jp];
+            if (page >= 0 && page < p.num_pages) nv = Lrow - jp * MLA_PAGE_SIZE;
+            else page = -1;
+          }
+          if constexpr (kFp8) {
+            // the page's per-token scales, published by the barrier below
+            if (i < 64) st_shared_u32(scl + 4u * uint32_t(i), __float_as_uint(page >= 0 ? p.kv_scale[size_t(page) * 64 + i] : 0.f));
+          }
           if (!gwait(ctl, bar(bars->s_full), bc & 1u, g == 0)) return false;
           if (g == 0) MLA_TR(2, 1, bc);
           tc_fence_after();
-          uint32_t sv0[32], sv1[32];
-          tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
-          tmem_ld32(tmem + lane_off + kTmemS + 64u * h + 32u, sv1);
-          tmem_wait_ld();
+          float x[64];
+          {
+            uint32_t sv0[32], sv1[32];
+            if constexpr (kFp8) {
+              // S = scale_j * S_lat + S_rope: the e4m3 values are unscaled
+              tmem_ld32(tmem + lane_off + kTmemSLat + 64u * h, sv0);
+              tmem_ld32(tmem + lane_off + kTmemSLat + 64u * h + 32u, sv1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; c += 4) {
+                const uint4 s0 = ld_shared_v4(scl + 4u * uint32_t(c)), s1 = ld_shared_v4(scl + 128u + 4u * uint32_t(c));
+                x[c] = __uint_as_float(sv0[c]) * __uint_as_float(s0.x);
+                x[c + 1] = __uint_as_float(sv0[c + 1]) * __uint_as_float(s0.y);
+                x[c + 2] = __uint_as_float(sv0[c + 2]) * __uint_as_float(s0.z);
+                x[c + 3] = __uint_as_float(sv0[c + 3]) * __uint_as_float(s0.w);
+                x[c + 32] = __uint_as_float(sv1[c]) * __uint_as_float(s1.x);
+                x[c + 33] = __uint_as_float(sv1[c + 1]) * __uint_as_float(s1.y);
+                x[c + 34] = __uint_as_float(sv1[c + 2]) * __uint_as_float(s1.z);
+                x[c + 35] = __uint_as_float(sv1[c + 3]) * __uint_as_float(s1.w);
+              }
+              tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
+              tmem_ld32(tmem + lane_off + kTmemS + 64u * h + 32u, sv1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                x[c] += __uint_as_float(sv0[c]);
+                x[c + 32] += __uint_as_float(sv1[c]);
+              }
+            } else {
+              tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
+              tmem_ld32(tmem + lane_off + kTmemS + 64u * h + 32u, sv1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                x[c] = __uint_as_float(sv0[c]);
+                x[c + 32] = __uint_as_float(sv1[c]);
+              }
+            }
+          }
           tc_fence_before();
           mbar_arrive(bar(bars->s_empty));
-
-          const int jp = j + h;                      // this thread's page
-          int nv = 0;                                // its visible tokens here
-          if (jp < pc.p1) {
-            const int page = p.block_table[size_t(r) * sv.max_pages + jp];
-            if (page >= 0 && page < p.num_pages) nv = Lrow - jp * MLA_PAGE_SIZE;
-          }
-          float x[64];
           float mh = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            x[c] = c < nv ? __uint_as_float(sv0[c]) * p.scale_log2 : -INFINITY;
-            x[c + 32] = c + 32 < nv ? __uint_as_float(sv1[c]) * p.scale_log2 : -INFINITY;
+            x[c] = c < nv ? x[c] * p.scale_log2 : -INFINITY;
+            x[c + 32] = c + 32 < nv ? x[c + 32] * p.scale_log2 : -INFINITY;
             mh = fmaxf(mh, fmaxf(x[c], x[c + 32]));
           }
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(xmax + 4u * uint32_t(g)), "f"(mh) : "memory");
@@ -711,7 +975,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         return true;
       });
     } else if (warp == 0) {
-      if (lane == 0) {  // ---- V producer: the page's first 512 columns (8 boxes) per stage
+      // ---- V producer: the page's 512 latent columns per stage.  BF16 cache:
+      // 8 boxes of 64 columns.  FP8 cache: 4 e4m3 boxes of 128 columns into
+      // the upper half of the stage (the converters expand them in place).
+      if (lane == 0) {
         uint32_t vc = 0;
         each_piece(sv, [&](const Piece& pc) {
           const int r = pc.T / sv.tiles_per_req;
@@ -721,10 +988,16 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             int page = p.block_table[size_t(r) * sv.max_pages + j];
             if (page < 0 || page >= p.num_pages) page = 0;   // the converters zero it
             const uint32_t fb = bar(bars->v_loaded[vs]);
-            mbar_arrive_expect_tx(fb, kVStage);
             const uint32_t dst = sbase + kOffV + vs * kVStage;
+            if constexpr (kFp8) {
+              mbar_arrive_expect_tx(fb, kVStage / 2);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) tma_load_3d(dst + c * kBox, &pool_map, 64 * c, 0, page, fb);
+              for (int c = 0; c < 4; ++c) tma_load_3d(dst + kVStage / 2 + c * kBox, &pool_map, 128 * c, 0, page, fb);
+            } else {
+              mbar_arrive_expect_tx(fb, kVStage);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) tma_load_3d(dst + c * kBox, &pool_map, 64 * c, 0, page, fb);
+            }
           }
           return true;
         });
@@ -749,19 +1022,55 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const int page = p.block_table[size_t(r) * sv.max_pages + j];
           const bool ok = page >= 0 && page < p.num_pages;
           const int nvalid = ok ? t - j * MLA_PAGE_SIZE : 0;
-          if (!wwait(ctl, bar(bars->v_loaded[vs]), vph)) return false;
-          if (ct == 0) MLA_TR(3, 1, vc);
           const uint32_t st = sbase + kOffV + vs * kVStage;
+          if constexpr (kFp8) {
+            // FP8 cache: output chunk o = ct + 256u (8 fp16 of token rr, in
+            // the N-major swizzled layout) comes from 8 e4m3 bytes of the
+            // upper half, times the token's scale.  The input and output
+            // regions overlap: every thread reads all its input before any
+            // thread writes.  Thread ct's chunks belong to tokens ct/8 and
+            // ct/8 + 32.
+            const int ta = ct >> 3;
+            const float sa = ok ? p.kv_scale[size_t(page) * 64 + ta] : 0.f;
+            const float sb = ok ? p.kv_scale[size_t(page) * 64 + ta + 32] : 0.f;
+            const bool vwait = ct == 0 ? bwait(ctl, bar(bars->v_loaded[vs]), vph) : true;
+            if (!named_bar_and(kConvBar, kConvThreads, vwait)) return false;
+            if (ct == 0) MLA_TR(3, 1, vc);
+            uint2 in[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
-            const int tok = int((off & (kBox - 1)) >> 7);
-            const uint4 v = ld_shared_v4(st + off);
-            if (tok < nvalid)
-              st_shared_v4(st + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                           bf16x2_to_f16x2(v.w));
-            else
-              st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+            for (int u = 0; u < 16; ++u) {
+              const uint32_t o = uint32_t(ct + kConvThreads * u), b = o >> 9, rr = (o & 511u) >> 3;
+              const uint32_t lc = (o & 7u) ^ (rr & 7u), k = 4u * (b & 1u) + (lc >> 1);
+              in[u] = ld_shared_v2(st + kVStage / 2 + (b >> 1) * kBox + rr * 128u + ((k ^ (rr & 7u)) << 4) +
+                                   (lc & 1u) * 8u);
+            }
+            named_bar_sync(kConvBar, kConvThreads);
+            const __half2 ha = __float2half2_rn(sa), hb = __float2half2_rn(sb);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const uint32_t o = uint32_t(ct + kConvThreads * u), rr = (o & 511u) >> 3;
+              if (int(rr) < nvalid) {
+                const __half2 sc = (u & 1) ? hb : ha;
+                st_shared_v4(st + o * 16u, e4m3x2_scaled(in[u].x & 0xFFFFu, sc), e4m3x2_scaled(in[u].x >> 16, sc),
+                             e4m3x2_scaled(in[u].y & 0xFFFFu, sc), e4m3x2_scaled(in[u].y >> 16, sc));
+              } else {
+                st_shared_v4(st + o * 16u, 0u, 0u, 0u, 0u);
+              }
+            }
+          } else {
+            if (!wwait(ctl, bar(bars->v_loaded[vs]), vph)) return false;
+            if (ct == 0) MLA_TR(3, 1, vc);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+              const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
+              const int tok = int((off & (kBox - 1)) >> 7);
+              const uint4 v = ld_shared_v4(st + off);
+              if (tok < nvalid)
+                st_shared_v4(st + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
+                             bf16x2_to_f16x2(v.w));
+              else
+                st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+            }
           }
           fence_proxy_async_cta();
           mbar_arrive(bar(bars->v_full[vs]));
@@ -811,6 +1120,32 @@ bool make_pool_map(CUtensorMap* map, const void* kv, int num_pages) {
   return r == CUDA_SUCCESS;
 }
 
+// FP8 cache pages [pages][40960 B]: the e4m3 latent block viewed as
+// [pages][64 tokens][512 bytes] with boxes of 128 bytes (columns) x 64
+// tokens, and the bf16 RoPE block (at +32 KB in each page) viewed as
+// [pages][64 tokens][64] with boxes of 64 columns x 64 tokens; both with the
+// 128-byte swizzle.
+bool make_fp8_maps(CUtensorMap* lat, CUtensorMap* rope, const void* kv, int num_pages) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dl[3] = {512, cuuint64_t(MLA_PAGE_SIZE), cuuint64_t(num_pages)};
+  cuuint64_t sl[2] = {512, kFp8PageBytes};
+  cuuint32_t bl[3] = {128, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(lat, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kv), dl, sl, bl, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  cuuint64_t dr[3] = {64, cuuint64_t(MLA_PAGE_SIZE), cuuint64_t(num_pages)};
+  cuuint64_t sr[2] = {128, kFp8PageBytes};
+  cuuint32_t br[3] = {64, 64, 1};
+  r = fn(rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+         const_cast<uint8_t*>(static_cast<const uint8_t*>(kv)) + 64 * 512, dr, sr, br, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over the query rows [batch * s_q * heads][576] bf16: boxes of
 // 64 columns x 64 rows, 128-byte swizzle.  Rows past the end read as zero.
 bool make_q_map(CUtensorMap* map, const void* q, int rows) {
@@ -839,23 +1174,30 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (shape->cache_dtype != MLA_CACHE_BF16) {
-    cudaError_t e = launch_decode_simt(q, kv, kv_scale, block_table, seqlens, scale, sched, ws, out, lse,
-                                       shape->num_pages, 1, cap_slots, sms, stream);
-    return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
-  }
+  const bool fp8 = shape->cache_dtype == MLA_CACHE_FP8_E4M3;
   const int q_rows = shape->batch * shape->s_q * shape->num_heads;
-  CUtensorMap pool_map, q_map;
-  if (!make_pool_map(&pool_map, kv, shape->num_pages) || !make_q_map(&q_map, q, q_rows)) return MLA_ERR_CUDA;
+  CUtensorMap pool_map, q_map, rope_map;
+  if (fp8) {
+    if (!make_fp8_maps(&pool_map, &rope_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+  } else {
+    if (!make_pool_map(&pool_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+    rope_map = pool_map;   // not read
+  }
+  if (!make_q_map(&q_map, q, q_rows)) return MLA_ERR_CUDA;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(decode_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    attr_err = cudaFuncSetAttribute(decode_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(kSmemBytes));
+    if (attr_err == cudaSuccess)
+      attr_err = cudaFuncSetAttribute(decode_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(kSmemBytes));
   });
   if (attr_err != cudaSuccess) return MLA_ERR_CUDA;
   Params prm;
   prm.q = static_cast<const uint16_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv);
+  prm.kv_scale = kv_scale;
   prm.block_table = block_table;
   prm.seqlens = seqlens;
   prm.sched = sched;
@@ -881,7 +1223,8 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_sm100_kernel, pool_map, q_map, prm);
+  const cudaError_t e = fp8 ? cudaLaunchKernelEx(&cfg, decode_sm100_kernel<true>, pool_map, q_map, rope_map, prm)
+                            : cudaLaunchKernelEx(&cfg, decode_sm100_kernel<false>, pool_map, q_map, rope_map, prm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
