@@ -198,6 +198,74 @@ def run_reference(args, wl, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
+    """Steps per unit time of the whole decode step including its host
+    transfers, pipelined over three streams (upload, compute, download)."""
+    import mla_latent_space_b200 as mla
+    nbuf = 2
+    h_q = wl.q.pin_memory()
+    h_bt = torch.from_numpy(wl.block_table).pin_memory()
+    h_sl = torch.from_numpy(wl.seqlens).pin_memory()
+    oshape = (wl.batch, wl.s_q, wl.num_heads, 512)
+    lshape = (wl.batch, wl.s_q, wl.num_heads)
+    h_out = [torch.empty(oshape, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    h_lse = [torch.empty(lshape, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    d_q = [torch.empty_like(h_q, device=dev) for _ in range(nbuf)]
+    d_bt = [torch.empty_like(h_bt, device=dev) for _ in range(nbuf)]
+    d_sl = [torch.empty_like(h_sl, device=dev) for _ in range(nbuf)]
+    d_out = [torch.empty(oshape, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
+    d_lse = [torch.empty(lshape, dtype=torch.float32, device=dev) for _ in range(nbuf)]
+    decs = [mla.Decoder(shape, device=dev) for _ in range(nbuf)]
+    s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    up_done = [ev() for _ in range(nbuf)]
+    comp_done = [ev() for _ in range(nbuf)]
+    down_done = [ev() for _ in range(nbuf)]
+    used = [False] * nbuf
+
+    def step(k):
+        b = k % nbuf
+        with torch.cuda.stream(s_up):
+            if used[b]:
+                s_up.wait_event(down_done[b])       # its previous step is downloaded (so computed)
+            d_q[b].copy_(h_q, non_blocking=True)
+            d_bt[b].copy_(h_bt, non_blocking=True)
+            d_sl[b].copy_(h_sl, non_blocking=True)
+            up_done[b].record(s_up)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(up_done[b])
+            decs[b].schedule(d_sl[b], stream=s_comp)
+            decs[b].decode(d_q[b], pool, kv_scale, d_bt[b], d_sl[b], wl.softmax_scale, d_out[b], d_lse[b],
+                           stream=s_comp)
+            comp_done[b].record(s_comp)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(comp_done[b])
+            h_out[b].copy_(d_out[b], non_blocking=True)
+            h_lse[b].copy_(d_lse[b], non_blocking=True)
+            down_done[b].record(s_down)
+        used[b] = True
+
+    for k in range(max(3, args.warmup)):
+        step(k)
+    torch.cuda.synchronize()
+    for dd in decs:
+        st = dd.status()
+        if st != 0:
+            raise RuntimeError(f"device status in the end-to-end loop: {mla.error_string(st)}")
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(s_up)
+    for k in range(K):
+        step(k)
+    s_up.wait_stream(s_down)
+    t1.record(s_up)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(t0.elapsed_time(t1) / K, world)
+
+
 def run_ours(args, wl, world, rank, local):
     import mla_latent_space_b200 as mla
     from mla_latent_space_b200 import build
@@ -267,38 +335,17 @@ def run_ours(args, wl, world, rank, local):
     if st != 0:
         raise RuntimeError(f"device status after timing: {mla.error_string(st)}")
 
-    # end to end through the public API with host buffers: per step the
-    # query, block table and lengths go host->device, the output and lse
-    # come back device->host (the KV cache is resident device state)
-    h_q = wl.q.pin_memory()
-    h_bt = torch.from_numpy(wl.block_table).pin_memory()
-    h_sl = torch.from_numpy(wl.seqlens).pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h2d = h_q.numel() * 2 + h_bt.numel() * 4 + h_sl.numel() * 4
-    d2h = h_out.numel() * 2 + h_lse.numel() * 4
-
-    def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        bt.copy_(h_bt, non_blocking=True)
-        sl.copy_(h_sl, non_blocking=True)
-        step()
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
-
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
-    torch.cuda.synchronize()
-    ev_e2e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    barrier(world)
-    for k in range(K):
-        flush.zero_()
-        ev_e2e[k][0].record(stream)
-        e2e_step()
-        ev_e2e[k][1].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev_e2e) / K, world)
+    # End to end through the public API with host buffers.  Every step copies
+    # its query, block table and lengths host -> device (pinned memory) and
+    # its output and lse device -> host; the KV cache is resident device
+    # state.  The steps run as a serving loop would: the copies go on their
+    # own streams with double-buffered device tensors, so step k's kernels
+    # overlap step k+1's upload and step k-1's download (a step's kernels
+    # wait for its upload; a buffer is reused only after the step that last
+    # used it has been downloaded).  The cache (302 MB) is larger than L2.
+    e2e_ms = run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world)
+    h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
+    d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
 
     flops, nbytes = cost.workload_cost(wl)
     pk, pk_kind = peaks()
@@ -335,7 +382,8 @@ def run_ours(args, wl, world, rank, local):
             "roofline": roof,
             "clocks": clk,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "pipelining": "upload / compute / download streams, 2 buffers"},
             "gpu_launches": 3 * K}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10 s of oracle work: the sample repeated until 10 s have passed
