@@ -78,7 +78,6 @@ MLA_HD int tile_pages(const ShapeInfo& s, int t, int qt) {
 }
 
 MLA_HD int tile_cost(int pages) { return pages > 0 ? pages + kPieceOverhead : 0; }
-
 // Last index i in [0, n) with a[i*stride] <= x (a non-decreasing); -1 if none.
 MLA_HD int last_le(const int32_t* a, int stride, int n, int64_t x) {
   int lo = 0, hi = n;  // answer in [lo-1, hi-1]
@@ -91,5 +90,28 @@ MLA_HD int last_le(const int32_t* a, int stride, int n, int64_t x) {
 
 // Lexicographic (tile, page) key.
 MLA_HD int64_t tp_key(int tile, int page) { return (int64_t(tile) << 32) | uint32_t(page); }
+
+// Extra cost, in page units, of a tile finished through fp32 partials: its
+// pieces' 128x512 fp32 writes and reads and the combine launch.  The
+// scheduler cuts tiles only when the whole-tile assignment's longest worker
+// exceeds the even share by more than this.  (Measured on B200: 64 equal
+// 64-page tiles over 74 SM pairs run faster whole, 1 tile per worker, than
+// cut to the even share of 57 units.)
+constexpr int kSplitOverhead = 12;
+
+// Whole-tile assignment: worker w of We takes the tiles whose cost prefix
+// lies in [total*w/We, total*(w+1)/We).  prefix[T*stride] is tile T's
+// exclusive cost prefix (non-decreasing); the range is [*tb, *te).
+MLA_HD void whole_tile_range(const int32_t* prefix, int stride, int num_tiles, int64_t total, int64_t We, int w,
+                             int* tb, int* te) {
+  if (w >= We) { *tb = *te = num_tiles; return; }
+  const int64_t x0 = total * w / We, x1 = total * (w + 1) / We;
+  *tb = last_le(prefix, stride, num_tiles, x0 - 1) + 1;
+  *te = w + 1 < We ? last_le(prefix, stride, num_tiles, x1 - 1) + 1 : num_tiles;
+}
+
+MLA_HD int64_t prefix_at(const int32_t* prefix, int stride, int num_tiles, int64_t total, int T) {
+  return T < num_tiles ? int64_t(prefix[size_t(T) * stride]) : total;
+}
 
 }  // namespace mla

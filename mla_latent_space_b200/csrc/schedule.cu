@@ -12,6 +12,12 @@
 // combine kernel merges.  This replaces the pages' radix-sorted block
 // scheduler with a prefix sum and binary searches: the same balance for a
 // contiguous assignment, and every step is parallel.
+//
+// Cutting a tile costs its pieces' fp32 partials and the combine, so the
+// scheduler first prices the whole-tile assignment (worker boundaries moved
+// to tile starts, whole_tile_range) and keeps it when its longest worker is
+// within kSplitOverhead of the even share: batches of similar lengths then
+// run without partials, jagged ones are cut.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -104,6 +110,23 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* warp_tot, int64_t* e
   return total;
 }
 
+// Block-wide maximum of one int64 per thread.
+__device__ int64_t block_max(int64_t v, int64_t* warp_tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const int64_t u = __shfl_xor_sync(0xffffffffu, v, off);
+    v = u > v ? u : v;
+  }
+  if (lane == 0) warp_tot[warp] = v;
+  __syncthreads();
+  int64_t m = 0;
+#pragma unroll
+  for (int k = 0; k < kSchedWarps; ++k) m = warp_tot[k] > m ? warp_tot[k] : m;
+  __syncthreads();
+  return m;
+}
+
 // First index in [0, W) whose key is >= key (keys non-decreasing).
 __device__ __forceinline__ int first_key_ge(const int64_t* keys, int W, int64_t key) {
   int lo = 0, hi = W;
@@ -159,8 +182,42 @@ schedule_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t
   }
   __syncthreads();
 
-  // 3: worker start positions (only min(W, total) workers get work)
+  // whole tiles or cut tiles: the whole-tile assignment's longest worker
   const int64_t We = total < W ? total : W;
+  int64_t mw = 0;
+  for (int w = tid; w < We; w += kSchedThreads) {
+    int tb, te;
+    whole_tile_range(prefix_sm, 1, num_tiles, total, We, w, &tb, &te);
+    const int64_t c = prefix_at(prefix_sm, 1, num_tiles, total, te) - prefix_at(prefix_sm, 1, num_tiles, total, tb);
+    mw = c > mw ? c : mw;
+  }
+  mw = block_max(mw, warp_tot);
+  const bool whole = We > 0 && mw <= (total + We - 1) / We + kSplitOverhead;
+  if (whole) {
+    for (int w = tid; w < W; w += kSchedThreads) {
+      int tb, te;
+      whole_tile_range(prefix_sm, 1, num_tiles, total, We, w, &tb, &te);
+      int32_t* wm = workers + size_t(w) * kWorkerInts;
+      wm[W_TILE_BEGIN] = tb;
+      wm[W_PAGE_BEGIN] = 0;
+      wm[W_TILE_END] = te;
+      wm[W_PAGE_END] = 0;
+      for (int k = W_FIRST_SPLIT; k < kWorkerInts; ++k) wm[k] = 0;
+    }
+    for (int T = t0; T < t1; ++T) {
+      tiles[size_t(T) * kTileInts + T_SPLITS] = pages_sm[T] > 0 ? 1 : 0;
+      tiles[size_t(T) * kTileInts + T_SLOT_BASE] = 0;
+    }
+    if (tid == 0) {
+      fill_header(hdr, s, W, num_tiles);
+      hdr[H_TOTAL_COST] = int32_t(total);
+      hdr[H_MAX_SLOTS] = 0;
+      hdr[H_STATUS] = flag_sh;
+    }
+    return;
+  }
+
+  // 3: worker start positions (only min(W, total) workers get work)
   for (int w = tid; w < W; w += kSchedThreads) {
     int tile = num_tiles, page = 0;
     if (w < We) {
@@ -228,6 +285,39 @@ MLA_HD void plan_schedule_seq(const int32_t* seqlens, const ShapeInfo& s, int W,
     tiles[size_t(T) * kTileInts + T_PAGES] = pages;
     tiles[size_t(T) * kTileInts + T_PREFIX] = int32_t(total);
     total += tile_cost(pages);
+  }
+  {
+    const int64_t We = total < W ? total : W;
+    const int32_t* prefix = tiles + T_PREFIX;
+    int64_t mw = 0;
+    for (int w = 0; w < We; ++w) {
+      int tb, te;
+      whole_tile_range(prefix, kTileInts, num_tiles, total, We, w, &tb, &te);
+      const int64_t c = prefix_at(prefix, kTileInts, num_tiles, total, te) -
+                        prefix_at(prefix, kTileInts, num_tiles, total, tb);
+      mw = c > mw ? c : mw;
+    }
+    if (We > 0 && mw <= (total + We - 1) / We + kSplitOverhead) {
+      for (int w = 0; w < W; ++w) {
+        int tb, te;
+        whole_tile_range(prefix, kTileInts, num_tiles, total, We, w, &tb, &te);
+        int32_t* wm = workers + size_t(w) * kWorkerInts;
+        wm[W_TILE_BEGIN] = tb;
+        wm[W_PAGE_BEGIN] = 0;
+        wm[W_TILE_END] = te;
+        wm[W_PAGE_END] = 0;
+        for (int k = W_FIRST_SPLIT; k < kWorkerInts; ++k) wm[k] = 0;
+      }
+      for (int T = 0; T < num_tiles; ++T) {
+        tiles[size_t(T) * kTileInts + T_SPLITS] = tiles[size_t(T) * kTileInts + T_PAGES] > 0 ? 1 : 0;
+        tiles[size_t(T) * kTileInts + T_SLOT_BASE] = 0;
+      }
+      fill_header(hdr, s, W, num_tiles);
+      hdr[H_TOTAL_COST] = int32_t(total);
+      hdr[H_MAX_SLOTS] = 0;
+      hdr[H_STATUS] = flag;
+      return;
+    }
   }
   for (int w = 0; w < W; ++w) {
     int tile, page;

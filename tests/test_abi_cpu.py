@@ -175,13 +175,33 @@ def check_schedule(seqlens, s_q, h, causal, n_sms):
     for T in range(b * tpr):
         if sc["tiles"][T, 0] == 0:
             assert sc["tiles"][T, 2] == 0
-    # balance: no worker exceeds the even share by more than one piece's overhead + 1 page
+    # balance.  Cut tiles: no worker exceeds the even share by more than one
+    # piece's overhead + 1 page.  Whole tiles (chosen when no tile needs
+    # cutting): the longest worker is within the split overhead (12 pages) of
+    # the even share over the workers that get work.
     cost = np.zeros(W)
     for w, T, p0, p1, split in pcs:
         cost[w] += (p1 - p0) + 2
     total = sc["hdr"][4]
-    assert cost.max() <= total / W + 2 * 2 + 1
+    if (sc["tiles"][:, 2] > 1).any():
+        assert cost.max() <= total / W + 2 * 2 + 1
+    elif total > 0:
+        We = min(W, total)
+        assert cost.max() <= -(-total // We) + 12
+        assert sc["hdr"][5] == 0 and all(p0 == 0 for _, _, p0, _, _ in pcs)
     return sc
+
+
+def test_schedule_chooses_whole_tiles_for_similar_lengths():
+    """64 requests of 4096 tokens on 74 SM pairs: cutting every tile to the
+    even share (57 units) saves less than partials + combine cost, so every
+    tile stays whole; the jagged batch is cut."""
+    sc = check_schedule([4096] * 64, 1, 128, False, 148)
+    assert (sc["tiles"][:, 2] == 1).all() and sc["hdr"][5] == 0
+    import mla_workloads as mw
+    _, _, _, lens = mw.config_shape(3)
+    sc = check_schedule(list(lens), 1, 128, False, 148)
+    assert (sc["tiles"][:, 2] > 1).any() and sc["hdr"][5] > 0
 
 
 @pytest.mark.parametrize("n_sms", [2, 3, 8, 148, 300])
