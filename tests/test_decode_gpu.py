@@ -101,3 +101,41 @@ def test_bad_page_id_is_flagged_not_faulted():
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 def test_full_size_configs_sampled(cfg):
     check_sampled(mw.make_config(cfg), n=4)
+
+
+# ---- FP8 cache: the kFp8 kernel across the same edge cases ------------------
+
+def test_fp8_causal_spec_and_packed_tiles():
+    check_full(mw.make(3, 16, 128, [200, 16, 700], causal=True, cache_dtype="fp8", seed=13, name="fp8_spec"))
+    check_full(mw.make(3, 2, 64, [130, 5, 260], causal=True, cache_dtype="fp8", seed=14, name="fp8_h64s2"))
+
+
+@pytest.mark.parametrize("n_sms", [2, 16, 1000])
+def test_fp8_split_counts_agree(n_sms):
+    wl = mw.make(4, 1, 128, [3000, 64, 1, 2500], cache_dtype="fp8", seed=15, name="fp8_splits")
+    check_full(wl, n_sms=n_sms)
+
+
+def test_fp8_nan_in_unused_slots_and_pages():
+    """e4m3 NaN bytes, bf16 NaN RoPE values and NaN scales past each
+    request's length, and unused block-table slots pointing at NaN pages,
+    change nothing."""
+    wl = mw.make(3, 1, 128, [70, 130, 1], cache_dtype="fp8", seed=16, name="fp8_poison")
+    O0, L0, _ = run(wl)
+    pool = wl.pool.clone()
+    scale = wl.kv_scale.clone()
+    nan_bf16 = torch.tensor([float("nan")], dtype=torch.bfloat16).view(torch.uint8)   # 2 bytes
+    for r, t in enumerate(wl.seqlens):
+        n = (int(t) + 63) // 64
+        last = int(wl.block_table[r, n - 1])
+        for tok in range(int(t) % 64 if t % 64 else 64, 64):
+            pool[last, tok * 512:(tok + 1) * 512] = 0x7F                       # e4m3 NaN
+            rope = pool[last, 64 * 512 + tok * 128:64 * 512 + (tok + 1) * 128].view(-1, 2)
+            rope[:] = nan_bf16
+            scale[last, tok] = float("nan")
+        wl.block_table[r, n:] = wl.num_pages                                   # the extra NaN page
+    extra = torch.full((1, pool.shape[1]), 0x7F, dtype=torch.uint8)
+    wl.pool = torch.cat([pool, extra])
+    wl.kv_scale = torch.cat([scale, torch.full((1, 64), float("nan"))])
+    O1, L1, st = run(wl)
+    assert st == 0 and np.isfinite(O1).all() and np.array_equal(O0, O1) and np.array_equal(L0, L1)
