@@ -57,7 +57,11 @@ using namespace ptx;
 constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring (bf16 cache)
 constexpr int NZ8 = 6;  // the same ring for the FP8 cache (e4m3 and RoPE stages)
 constexpr int NC = 4;   // FP8 cache: 16 KB stages of fp16 cache rows converted from e4m3
-constexpr int NX = 1;   // P block stages (output CTA)
+// P page slots (output CTA): slot 0 takes page 0 of a block with the block's
+// rescale factors and row sums, slot 1 its page 1.  Each is refilled as soon
+// as its own page's PVs completed, so the next block's page 0 crosses over
+// while this block's page 1 is multiplied.
+constexpr int NX = 2;
 constexpr int NV = 3;   // V page stages (output CTA): its own TMA ring
 // Per-block PV completion barriers for the correction warpgroup.  It may lag
 // the MMAs by up to three blocks (a block's P arrives once PV of block - 2
@@ -73,11 +77,13 @@ constexpr uint32_t kBox = 8192;                       // 64 rows x 128 B
 constexpr uint32_t kZStage = 2 * kBox;                // one 64-column box of both pages (128 rows)
 constexpr uint32_t kPageBytes = 9 * kBox;             // 64 tokens x 576 bf16
 constexpr uint32_t kVStage = 8 * kBox;                // 64 tokens x 512 fp16
-constexpr uint32_t kPBytes = 2 * 128 * 128;           // 128 rows x 128 fp16 (two pages)
+constexpr uint32_t kPPage = 128 * 64 * 2;             // 128 rows x 64 fp16 (one page of P)
 constexpr uint32_t kMetaBytes = 1024;                 // alpha[128], l[128]
-constexpr uint32_t kPStage = kPBytes + kMetaBytes;    // one bulk copy per block
+constexpr uint32_t kPSlot0 = kPPage + kMetaBytes;     // page 0 and the block's meta
+constexpr uint32_t kPStage = kPSlot0 + kPPage;        // both slots; also the score CTA's staging
 constexpr uint32_t kTmemS = 384;                      // S accumulator: columns 384..511
-constexpr uint64_t kTimeoutNs = 2000000000ull;        // a wait gives up after 2 s
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kEvRescale = 1, kEvEnd = 2;        // correction events (Bars::ev_type)        // a wait gives up after 2 s
 constexpr float kLazyMax = 8.0f;                      // log2 units
 constexpr int kConvThreads = 256;                     // output-CTA warps 8..15
 constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
@@ -92,7 +98,12 @@ struct Bars {
   uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
   uint64_t c_full[NC], c_empty[NC], qpe_full, qpe_empty;
   // output CTA
-  uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_done[NX], pv_blk[NB], o_free;
+  uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_go, corr_done, pv_blk[NB], o_free;
+  // correction events, from the PV issuer warp to the correction warpgroup:
+  // a block's rescale factors (O must be rescaled before its PVs) or, at the
+  // end of a piece, its row sums (normalise and store O)
+  uint32_t ev_type, ev_blk;
+  alignas(16) float ev_val[128];
   // both
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -119,11 +130,12 @@ constexpr uint32_t kSmemS = LayS<false>::end > LayS<true>::end ? LayS<false>::en
 // output CTA
 constexpr uint32_t kOffV = kOffData;
 constexpr uint32_t kOffP = kOffV + NV * kVStage;              // P + meta block stages
-constexpr uint32_t kSmemO = kOffP + NX * kPStage;
+constexpr uint32_t kSmemO = kOffP + kPStage;
 constexpr uint32_t kSmemBytes = (kSmemS > kSmemO ? kSmemS : kSmemO) + 1024;  // + alignment slack
 static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kPStage % 1024 == 0 && kZStage % 1024 == 0, "swizzle atoms need 1024-byte alignment");
+static_assert(kPSlot0 % 1024 == 0 && kPStage % 1024 == 0 && kZStage % 1024 == 0,
+              "swizzle atoms need 1024-byte alignment");
 static_assert(LayS<true>::c % 1024 == 0 && LayS<true>::qpe % 1024 == 0 && LayS<true>::stage % 1024 == 0, "align");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
@@ -252,13 +264,34 @@ __device__ __forceinline__ bool wwait(const Ctl& c, uint32_t bar, uint32_t parit
   return ok;
 }
 
+// Issuer-warp bounded wait: every lane polls without suspending (each lane
+// holds its own acquire) and the warp leaves together.
+template <bool kCluster = false>
+__device__ __forceinline__ bool ewait(const Ctl& c, uint32_t bar, uint32_t parity) {
+  auto once = [&] { return kCluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity); };
+  if (__all_sync(0xffffffffu, once())) return true;
+  const bool lead = (threadIdx.x & 31) == 0;
+  const uint64_t t0 = lead ? globaltimer() : 0ull;
+  for (uint32_t n = 1;; ++n) {
+    if (__all_sync(0xffffffffu, once())) return true;
+    if ((n & 15) == 0) {
+      const int stop = __shfl_sync(0xffffffffu, lead ? (*c.abort ? 1 : (globaltimer() - t0 > kTimeoutNs ? 2 : 0)) : 0, 0);
+      if (stop != 0) {
+        if (stop == 2 && lead) trip(c);
+        return false;
+      }
+    }
+  }
+}
+
 // Softmax-group bounded wait: the group's first thread polls, the named
 // barrier hands its verdict (and, through the barrier, its acquire) to the
 // other 255 threads, and the group decides together (a thread leaving alone
-// would strand the others at the group's named barrier).
-__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity, bool poller) {
+// would strand the others at the group's named barrier).  `carried` is the
+// poller's verdict on an earlier wait the group did not wait for.
+__device__ __forceinline__ bool gwait(const Ctl& c, uint32_t bar, uint32_t parity, bool poller, bool carried = true) {
   bool ok = true;
-  if (poller) ok = bwait(c, bar, parity);
+  if (poller) ok = carried && bwait(c, bar, parity);
   return named_bar_and(kSoftmaxBar, kSmThreads, ok);
 }
 
@@ -360,8 +393,9 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     for (int s = 0; s < NX; ++s) {
       mbar_init(bar(bars->x_free[s]), 1);
       mbar_init(bar(bars->p_full[s]), 1);
-      mbar_init(bar(bars->corr_done[s]), 128);
     }
+    mbar_init(bar(bars->corr_go), 32);
+    mbar_init(bar(bars->corr_done), 128);
     for (int s = 0; s < NV; ++s) {
       mbar_init(bar(bars->v_loaded[s]), 1);
       mbar_init(bar(bars->v_full[s]), kConvThreads);
@@ -379,9 +413,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     bars->abort = 0;
     for (int k = 0; k < 8; ++k) bars->trc[k] = 0;
     fence_mbar_init();
-    // the output CTA arms its P stages for their first bulk copy
-    if (rank == 1)
-      for (int s = 0; s < NX; ++s) mbar_arrive_expect_tx(bar(bars->p_full[s]), kPStage);
+    // the output CTA arms its P slots for their first bulk copies
+    if (rank == 1) {
+      mbar_arrive_expect_tx(bar(bars->p_full[0]), kPSlot0);
+      mbar_arrive_expect_tx(bar(bars->p_full[1]), kPPage);
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&pool_map);
@@ -498,99 +534,117 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         if (kFp8 && pieces > 0) drain_wait(bar(bars->qpe_full), (pieces - 1) & 1u);
       }
     } else if (warp == 1) {
-      // ---- QK^T issuer: per block 36 MMAs M128 N128 K16.  BF16 cache: 9
+      // ---- QK^T issuer warp: per block 36 MMAs M128 N128 K16.  BF16 cache: 9
       // stages x 4, A = Q (TMEM), into S.  FP8 cache: the RoPE stage x 4 with
       // A = the query RoPE columns (shared memory) into S_rope, then 8
       // converted fp16 stages x 4 with A = the fp16 query (TMEM) into S_lat.
-      if (lane == 0) {
-        const uint64_t zdesc0 = sdesc(sbase + L::z, 16, 1024);
-        const uint64_t cdesc0 = sdesc(sbase + L::c, 16, 1024);
-        const uint64_t qdesc = sdesc(sbase + L::qpe, 16, 1024);
-        uint32_t zc = 0, cc = 0, bc = 0, pieces = 0;
-        each_piece(sv, [&](const Piece& pc) {
-          // FP8 cache: the ring is shorter than the query, so its stages are
-          // released one by one.  This thread and one converter thread walk
-          // every stage of the ring in order (a parity wait is only sound when
-          // the stage's previous use has completed), and a stage is refilled
-          // after three releases: softmax, issuer, converter.  For the RoPE
-          // and e4m3 stages, which the softmax never sees, the issuer releases
-          // twice.
-          constexpr int nq = kFp8 ? 8 : 9;
-          if constexpr (kFp8) {
-            for (int u = 0; u < nq; ++u, ++zc) {
-              if (!swait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
-              mbar_arrive(bar(bars->z_empty[zc % nz]));
-            }
+      // The warp waits and computes operands together; one lane issues.
+      const bool leader = elect_one();
+      const uint64_t zdesc0 = sdesc(sbase + L::z, 16, 1024);
+      const uint64_t cdesc0 = sdesc(sbase + L::c, 16, 1024);
+      const uint64_t qdesc = sdesc(sbase + L::qpe, 16, 1024);
+      uint32_t zc = 0, cc = 0, bc = 0, pieces = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        // FP8 cache: the ring is shorter than the query, so its stages are
+        // released one by one.  This warp and one converter thread walk
+        // every stage of the ring in order (a parity wait is only sound when
+        // the stage's previous use has completed), and a stage is refilled
+        // after three releases: softmax, issuer, converter.  For the RoPE
+        // and e4m3 stages, which the softmax never sees, the issuer releases
+        // twice.
+        constexpr int nq = kFp8 ? 8 : 9;
+        if constexpr (kFp8) {
+          for (int u = 0; u < nq; ++u, ++zc) {
+            if (!ewait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
+            if (leader) mbar_arrive(bar(bars->z_empty[zc % nz]));
           }
-          if (!swait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
-          if (kFp8 && !swait(ctl, bar(bars->qpe_full), pieces & 1u)) return false;
-          MLA_TR(1, 0, bc);
-          ++pieces;
-          // the query rows are in TMEM: release their stages
-          if constexpr (!kFp8) {
+        }
+        if (!ewait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
+        if (kFp8 && !ewait(ctl, bar(bars->qpe_full), pieces & 1u)) return false;
+        if (leader) MLA_TR(1, 0, bc);
+        ++pieces;
+        // the query rows are in TMEM: release their stages
+        if constexpr (!kFp8) {
+          if (leader)
             for (int u = 0; u < nq; ++u) mbar_arrive(bar(bars->z_empty[(zc + u) % nz]));
-            zc += nq;
-          }
+          zc += nq;
+        }
+        tc_fence_after();
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          if (!ewait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
+          if (leader) MLA_TR(1, 2, bc);
           tc_fence_after();
-          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-            if (!swait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
-            MLA_TR(1, 2, bc);
-            tc_fence_after();
-            if constexpr (kFp8) {
-              {
-                const uint32_t zs = zc % nz;
-                if (!swait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-                MLA_TR(1, 20, zc);
-                const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
-                const uint32_t d = tmem + kTmemS;
+          if constexpr (kFp8) {
+            {
+              const uint32_t zs = zc % nz;
+              if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
+              if (leader) MLA_TR(1, 20, zc);
+              tc_fence_after();
+              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+              const uint32_t d = tmem + kTmemS;
+              if (leader) {
                 mma_ss(d, qdesc, bd, kIdescQK, 0u);
                 mma_ss(d, qdesc + 2u, bd + 2u, kIdescQK, 1u);
                 mma_ss(d, qdesc + 4u, bd + 4u, kIdescQK, 1u);
                 mma_ss(d, qdesc + 6u, bd + 6u, kIdescQK, 1u);
                 mma_commit(bar(bars->z_empty[zs]));    // the issuer's release, when the MMAs are done
                 mbar_arrive(bar(bars->z_empty[zs]));   // the softmax's
+              }
+              __syncwarp();
+              ++zc;
+            }
+            for (int c = 0; c < 8; ++c, ++cc) {
+              if ((c & 1) == 0) {   // e4m3 stage c/2: observed in order, released for issuer and softmax
+                if (!ewait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
+                if (leader) mbar_arrive_cnt(bar(bars->z_empty[zc % nz]), 2u);
                 ++zc;
               }
-              for (int c = 0; c < 8; ++c, ++cc) {
-                if ((c & 1) == 0) {   // e4m3 stage c/2: observed in order, released for issuer and softmax
-                  if (!swait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
-                  mbar_arrive_cnt(bar(bars->z_empty[zc % nz]), 2u);
-                  ++zc;
-                }
-                const uint32_t cs = cc % NC;
-                if (!swait(ctl, bar(bars->c_full[cs]), (cc / NC) & 1u)) return false;
-                MLA_TR(1, 21, cc);
-                const uint64_t bd = cdesc0 + uint64_t(cs * (kZStage >> 4));
-                const uint32_t ad = tmem + 32u * c, d = tmem + kTmemSLat;
+              const uint32_t cs = cc % NC;
+              if (!ewait(ctl, bar(bars->c_full[cs]), (cc / NC) & 1u)) return false;
+              if (leader) MLA_TR(1, 21, cc);
+              tc_fence_after();
+              const uint64_t bd = cdesc0 + uint64_t(cs * (kZStage >> 4));
+              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemSLat;
+              if (leader) {
                 mma_ts(d, ad, bd, kIdescQKh, c != 0);
                 mma_ts(d, ad + 8u, bd + 2u, kIdescQKh, 1u);
                 mma_ts(d, ad + 16u, bd + 4u, kIdescQKh, 1u);
                 mma_ts(d, ad + 24u, bd + 6u, kIdescQKh, 1u);
                 mma_commit(bar(bars->c_empty[cs]));
               }
-            } else {
-              for (int c = 0; c < 9; ++c, ++zc) {
-                const uint32_t zs = zc % nz;
-                if (!swait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-                MLA_TR(1, 10 + c, bc);
-                const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
-                const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
+              __syncwarp();
+            }
+          } else {
+            for (int c = 0; c < 9; ++c, ++zc) {
+              const uint32_t zs = zc % nz;
+              if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
+              if (leader) MLA_TR(1, 10 + c, bc);
+              tc_fence_after();
+              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
+              if (leader) {
                 mma_ts(d, ad, bd, kIdescQK, c != 0);
                 mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
                 mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
                 mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
                 mma_commit(bar(bars->z_empty[zs]));
               }
+              __syncwarp();
             }
+          }
+          if (leader) {
             mma_commit(bar(bars->s_full));
             MLA_TR(1, 3, bc);
           }
-          if (kFp8) mma_commit(bar(bars->qpe_empty));   // the piece's RoPE MMAs are done with the buffer
-          return true;
-        });
-        mma_commit(bar(bars->mma_done));
-        drain_wait(bar(bars->mma_done), 0);
-      }
+          __syncwarp();
+        }
+        if (kFp8 && leader) mma_commit(bar(bars->qpe_empty));   // the piece's RoPE MMAs are done with the buffer
+        __syncwarp();
+        return true;
+      });
+      if (leader) mma_commit(bar(bars->mma_done));
+      __syncwarp();
+      drain_wait(bar(bars->mma_done), 0);
     } else if (kFp8 && warp >= 12) {
       // ---- FP8 cache: converters.  Each e4m3 stage (128 latent columns of
       // the block's two pages) becomes two fp16 stages of 64 columns in the
@@ -660,7 +714,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       const uint32_t stg = sbase + L::stage;
       const uint32_t xmax = sbase + L::xchg, xsum = xmax + 2 * 128 * 4;
       const uint32_t scl = sbase + L::scales + uint32_t(h) * 256;   // FP8: this page's 64 scales
-      uint32_t zc = 0, bc = 0;
+      uint32_t zc = 0, bc = 0, n1 = 0;   // n1: blocks with two pages so far (uses of slot 1)
+      bool carry_ok = true;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
@@ -681,7 +736,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 #pragma unroll 1
           for (int c = 0; c < nq; ++c) {
             const uint32_t idx = zc + c;
-            if (!gwait(ctl, bar(bars->z_full[idx % nz]), (idx / nz) & 1u, g == 0)) return false;
+            if (!gwait(ctl, bar(bars->z_full[idx % nz]), (idx / nz) & 1u, g == 0, carry_ok)) return false;
             // FP8 cache: every thread has passed the barrier, so the previous
             // query stage has been read: the producer may refill it
             if (kFp8 && c > 0 && g == 0) mbar_arrive(bar(bars->z_empty[(idx - 1) % nz]));
@@ -727,7 +782,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             // the page's per-token scales, published by the barrier below
             if (i < 64) st_shared_u32(scl + 4u * uint32_t(i), __float_as_uint(page >= 0 ? p.kv_scale[size_t(page) * 64 + i] : 0.f));
           }
-          if (!gwait(ctl, bar(bars->s_full), bc & 1u, g == 0)) return false;
+          if (!gwait(ctl, bar(bars->s_full), bc & 1u, g == 0, carry_ok)) return false;
           if (g == 0) MLA_TR(2, 1, bc);
           tc_fence_after();
           float x[64];
@@ -806,7 +861,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           const float ph = (s0 + s1) + (s2 + s3);
           asm volatile("st.shared.f32 [%0], %1;" ::"r"(xsum + 4u * uint32_t(g)), "f"(ph) : "memory");
-          const uint32_t prow = stg + uint32_t(h) * (kPBytes / 2) + (i >> 3) * 1024 + (i & 7) * 128;
+          const uint32_t prow = stg + uint32_t(h) * kPSlot0 + (i >> 3) * 1024 + (i & 7) * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             st_shared_v4(prow + ((uint32_t(k) ^ uint32_t(i & 7)) << 4), pack_f16(x[8 * k], x[8 * k + 1]),
@@ -817,21 +872,29 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           l = l * alpha + ph + ld_shared_f32(xsum + 4u * uint32_t(g ^ 128));
           m = m_new;
           if (h == 0) {
-            st_shared_u32(stg + kPBytes + 4 * i, __float_as_uint(need ? alpha : 1.f));
-            st_shared_u32(stg + kPBytes + 512 + 4 * i, __float_as_uint(l));
+            st_shared_u32(stg + kPPage + 4 * i, __float_as_uint(need ? alpha : 1.f));
+            st_shared_u32(stg + kPPage + 512 + 4 * i, __float_as_uint(l));
           }
           fence_proxy_async_cta();
-          // the output CTA's block stage is free once its PVs completed;
-          // the barrier also publishes every staging write to thread 0
-          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-          const bool free_ok = g == 0 ? bwait<true>(ctl, bar(bars->x_free[xs]), xph ^ 1u) : true;
-          if (!named_bar_and(kSoftmaxBar, kSmThreads, free_ok)) return false;
-          if (g == 0) MLA_TR(2, 2, bc);
+          // publishes every staging write to thread 0, which ships page 0
+          // (with the meta) and page 1 to the output CTA's slots, each once
+          // the PVs of the previous block's same page completed.  A failed
+          // wait is reported at the group's next barrier.
+          named_bar_sync(kSoftmaxBar, kSmThreads);
+          const bool two = j + 1 < pc.p1;
           if (g == 0) {
-            bulk_copy_to_peer(o_p + xs * kPStage, stg, kPStage, o_pfull + xs * 8);
+            bool ok = bwait<true>(ctl, bar(bars->x_free[0]), (bc & 1u) ^ 1u);
+            MLA_TR(2, 2, bc);
+            if (ok) bulk_copy_to_peer(o_p, stg, kPSlot0, o_pfull);
+            if (ok && two) {
+              ok = bwait<true>(ctl, bar(bars->x_free[1]), (n1 & 1u) ^ 1u);
+              if (ok) bulk_copy_to_peer(o_p + kPSlot0, stg + kPSlot0, kPPage, o_pfull + 8u);
+            }
             bulk_commit_group();
+            carry_ok = ok;
             MLA_TR(2, 3, bc);
           }
+          n1 += two ? 1u : 0u;
         }
         if (valid && h == 0) {
           const float lse_v = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -851,91 +914,133 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   } else {
     // ======================= output CTA =======================
     if (warp == 1) {
-      if (lane == 0) {  // ---- PV issuer: per block, per page 4 K-steps x 2 N halves
-        const uint64_t pdesc0 = sdesc(sbase + kOffP, 16, 1024);
-        const uint64_t vdesc0 = sdesc(sbase + kOffV, kBox, 1024);
-        uint32_t bc = 0, vc = 0, pieces = 0;
-        each_piece(sv, [&](const Piece& pc) {
-          if (pieces > 0 && !swait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
-          MLA_TR(4, 0, bc);
-          ++pieces;
-          for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-            const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-            if (!swait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
-            MLA_TR(4, 1, bc);
-            if (!swait(ctl, bar(bars->corr_done[xs]), xph)) return false;
-            MLA_TR(4, 2, bc);
-            // arm this stage for its next block (its copy can only start
-            // after this block's PVs complete, which needs corr_done above)
-            mbar_arrive_expect_tx(bar(bars->p_full[xs]), kPStage);
+      // ---- PV issuer warp: per block, per page 4 K-steps x 2 N halves.  One
+      // lane issues; the warp reads the block's rescale factors and hands
+      // them to the correction warpgroup only when one of them is not 1.
+      const bool leader = elect_one();
+      const uint64_t pdesc0 = sdesc(sbase + kOffP, 16, 1024);
+      const uint64_t vdesc0 = sdesc(sbase + kOffV, kBox, 1024);
+      const uint32_t meta = sbase + kOffP + kPPage + 16u * uint32_t(lane);   // alpha[4 lane..]; l at +512
+      const uint32_t evv = smem_u32(&bars->ev_val[0]) + 16u * uint32_t(lane);
+      uint32_t bc = 0, vc = 0, pieces = 0, n1 = 0, nr = 0;
+      each_piece(sv, [&](const Piece& pc) {
+        if (pieces > 0 && !ewait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
+        if (leader) MLA_TR(4, 0, bc);
+        ++pieces;
+        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
+          const bool two = j + 1 < pc.p1, last = j + 2 >= pc.p1;
+          if (!ewait<true>(ctl, bar(bars->p_full[0]), bc & 1u)) return false;
+          if (leader) MLA_TR(4, 1, bc);
+          const float4 a4 = ld_shared_f4(meta);
+          const float4 l4 = last ? ld_shared_f4(meta + 512u) : make_float4(0.f, 0.f, 0.f, 0.f);
+          // re-arm slot 0: its next copy starts only after this block's
+          // page-0 PVs complete
+          if (leader) mbar_arrive_expect_tx(bar(bars->p_full[0]), kPSlot0);
+          if (__any_sync(0xffffffffu, a4.x != 1.f || a4.y != 1.f || a4.z != 1.f || a4.w != 1.f)) {
+            // the running max moved: O is rescaled (once every earlier PV
+            // completed) before this block's PVs
+            st_shared_f4(evv, a4);
+            if (leader) {
+              bars->ev_type = kEvRescale;
+              bars->ev_blk = bc;
+            }
+            mbar_arrive(bar(bars->corr_go));
+            if (!ewait(ctl, bar(bars->corr_done), nr & 1u)) return false;
+            ++nr;
+          }
+          if (leader) MLA_TR(4, 2, bc);
+          for (int u = 0; u < (two ? 2 : 1); ++u, ++vc) {
+            if (u == 1) {
+              if (!ewait<true>(ctl, bar(bars->p_full[1]), n1 & 1u)) return false;
+              if (leader) mbar_arrive_expect_tx(bar(bars->p_full[1]), kPPage);
+            }
+            const uint32_t vs = vc % NV;
+            if (!ewait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
+            if (leader) MLA_TR(4, 3, vc);
             tc_fence_after();
-            const int np = min(2, pc.p1 - j);
-            for (int u = 0; u < np; ++u, ++vc) {
-              const uint32_t vs = vc % NV;
-              if (!swait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
-              MLA_TR(4, 3, vc);
-              const uint64_t ad = pdesc0 + uint64_t((xs * kPStage + uint32_t(u) * (kPBytes / 2)) >> 4);
-              const uint64_t bd = vdesc0 + uint64_t((vs * kVStage) >> 4);
-              const uint32_t acc0 = (j > pc.p0 || u > 0) ? 1u : 0u;
+            const uint64_t ad = pdesc0 + uint64_t((uint32_t(u) * kPSlot0) >> 4);
+            const uint64_t bd = vdesc0 + uint64_t((vs * kVStage) >> 4);
+            const uint32_t acc0 = (j > pc.p0 || u > 0) ? 1u : 0u;
+            if (leader) {
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 mma_ss(tmem, ad + 2u * k, bd + (2048u >> 4) * k, kIdescPV, k > 0 ? 1u : acc0);
                 mma_ss(tmem + 256u, ad + 2u * k, bd + ((4u * kBox + 2048u * k) >> 4), kIdescPV, k > 0 ? 1u : acc0);
               }
               mma_commit(bar(bars->pv_done[vs]));
+              mma_commit_mc(bar(bars->x_free[u]), uint16_t(1u));   // the score CTA may refill slot u
             }
+            __syncwarp();
+          }
+          n1 += two ? 1u : 0u;
+          if (leader) {
             mma_commit(bar(bars->pv_blk[bc % NB]));
             MLA_TR(4, 4, bc);
-            mma_commit_mc(bar(bars->x_free[xs]), uint16_t(1u));
           }
-          return true;
-        });
-        mma_commit(bar(bars->mma_done));
-        drain_wait(bar(bars->mma_done), 0);
-      }
+          __syncwarp();
+          if (last) {
+            // the piece's row sums, for the epilogue (which waits for these PVs)
+            st_shared_f4(evv, l4);
+            if (leader) {
+              bars->ev_type = kEvEnd;
+              bars->ev_blk = bc;
+            }
+            mbar_arrive(bar(bars->corr_go));
+          }
+        }
+        return true;
+      });
+      if (leader) mma_commit(bar(bars->mma_done));
+      __syncwarp();
+      drain_wait(bar(bars->mma_done), 0);
     } else if (warp >= 4 && warp < 8) {
-      // ---- correction / epilogue warpgroup: thread i owns row i of O
+      // ---- correction / epilogue warpgroup: thread i owns row i of O.  It
+      // acts on the PV issuer's events: a block whose rescale factors are not
+      // all 1 (rescale O once every earlier block's PVs completed) and the end
+      // of a piece (normalise O by the row sums and store it).  An event's
+      // data stays put until the issuer sees it handled (corr_done, o_free).
       const int i = tid - 128, wq = warp - 4;
       const uint32_t lane_off = uint32_t(wq * 32) << 16;
-      uint32_t bc = 0;
+      const volatile Bars* vb = bars;
+      uint32_t ne = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
         const int rho = qt * MLA_TILE_ROWS + i;
         const bool valid = rho < rows_total;
-        float lfin = 0.f;
-        for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
-          const uint32_t xs = bc % NX, xph = (bc / NX) & 1u;
-          if (!wwait<true>(ctl, bar(bars->p_full[xs]), xph)) return false;
-          if (i == 0) MLA_TR(5, 1, bc);
-          const volatile float* meta = reinterpret_cast<const volatile float*>(gbase + kOffP + xs * kPStage + kPBytes);
-          const float alpha = meta[i];
-          if (j + 2 >= pc.p1) lfin = meta[128 + i];
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        for (;;) {
+          if (!wwait(ctl, bar(bars->corr_go), ne & 1u)) return false;
+          ++ne;
+          const uint32_t type = vb->ev_type, eb = vb->ev_blk;
+          const float v = vb->ev_val[i];
+          if (i == 0) MLA_TR(5, 1, eb);
+          if (type == kEvRescale) {
             // O must hold every earlier block before it is rescaled (never
-            // the piece's first block, so bc - 1 exists)
-            const uint32_t pb = bc - 1;
+            // the piece's first block, so eb - 1 exists)
+            const uint32_t pb = eb - 1;
             if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
-            tc_fence_after();
+            if (__any_sync(0xffffffffu, v != 1.f)) {
+              tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 16; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_off + 32u * c, o);
-              tmem_wait_ld();
+              for (int c = 0; c < 16; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + 32u * c, o);
+                tmem_wait_ld();
 #pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-              tmem_st32(tmem + lane_off + 32u * c, o);
+                for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * v);
+                tmem_st32(tmem + lane_off + 32u * c, o);
+              }
+              tmem_wait_st();
             }
-            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(bars->corr_done));
+            continue;
           }
-          tc_fence_before();
-          mbar_arrive(bar(bars->corr_done[xs]));
-        }
-        // epilogue: wait for the piece's last block of PVs, normalise, store
-        {
-          const uint32_t pb = bc - 1;
+          // end of the piece: wait for its last block of PVs, normalise, store
+          const uint32_t pb = eb;
           if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
-          if (i == 0) MLA_TR(5, 5, bc);
+          if (i == 0) MLA_TR(5, 5, eb);
           tc_fence_after();
+          const float lfin = v;
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
           const bool whole = sv.tile_splits(pc.T) == 1;
           const int slot = whole ? 0 : sv.tile_slot_base(pc.T) + pc.split;
@@ -970,9 +1075,9 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           tc_fence_before();
           mbar_arrive(bar(bars->o_free));
-          if (i == 0) MLA_TR(5, 6, bc);
+          if (i == 0) MLA_TR(5, 6, eb);
+          return true;
         }
-        return true;
       });
     } else if (warp == 0) {
       // ---- V producer: the page's 512 latent columns per stage.  BF16 cache:
