@@ -85,7 +85,7 @@ constexpr uint32_t kTmemS = 384;                      // S accumulator: columns 
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kEvRescale = 1, kEvEnd = 2;        // correction events (Bars::ev_type)        // a wait gives up after 2 s
 constexpr float kLazyMax = 8.0f;                      // log2 units
-constexpr int kConvThreads = 256;                     // output-CTA warps 8..15
+constexpr int kConvThreads = 256;                     // output-CTA converter warps (conv_rank)
 constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
 constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of the softmax warps
 constexpr uint32_t kConvBar = 2;                      // named barrier of a CTA's converter warps
@@ -108,7 +108,6 @@ struct Bars {
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort;
-  uint32_t trc[8];   // trace event counters (MLA_TRACE builds)
 };
 
 constexpr uint32_t kOffData = 1024;
@@ -185,7 +184,7 @@ struct Params {
 #define MLA_TR(role, ev, j)                                                               \
   do {                                                                                    \
     if (p.trace && cluster_id_x() == MLA_TRACE_CLUSTER) {                                                 \
-      const unsigned k_ = bars->trc[role]++;                                              \
+      const unsigned k_ = trk_++;                                                         \
       if (k_ < 2047) {                                                                    \
         unsigned long long* e_ = p.trace + (size_t(role) * 2048 + k_) * 3;                \
         e_[0] = (unsigned long long)(((ev) << 24) | (unsigned(j) & 0xFFFFFF));            \
@@ -346,6 +345,23 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   return v;
 }
 
+// Output CTA: the eight converter warps (-1 for other warps).  None shares a
+// scheduler sub-partition (warp % 4) with the PV issuer (warp 1): their
+// bursts of shared-memory loads would delay the issuer's barrier polls.
+__device__ __forceinline__ int conv_rank(int warp) {
+  switch (warp) {
+    case 2: return 0;
+    case 3: return 1;
+    case 8: return 2;
+    case 10: return 3;
+    case 11: return 4;
+    case 12: return 5;
+    case 14: return 6;
+    case 15: return 7;
+    default: return -1;
+  }
+}
+
 // Calls f(piece) for every piece of every worker this cluster owns; stops
 // when f returns false.
 template <class F>
@@ -379,6 +395,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
+  [[maybe_unused]] unsigned trk_ = 0;   // trace builds: this thread's event count (one recording thread per role)
 
   if (tid == 0) {
     // FP8 cache: a ring stage is refilled once the softmax, the issuer and
@@ -411,7 +428,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
-    for (int k = 0; k < 8; ++k) bars->trc[k] = 0;
     fence_mbar_init();
     // the output CTA arms its P slots for their first bulk copies
     if (rank == 1) {
@@ -448,11 +464,15 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     using L = LayS<kFp8>;
     constexpr int nz = L::nz;
     if (warp == 0) {
-      // ---- TMA producer.  BF16 cache: 9 query stages per piece, then 9 per
-      // 2-page block.  FP8 cache: 8 query stages (latent columns) plus the
-      // query RoPE columns into their own buffer per piece, then per block one
-      // RoPE stage (bf16) and 4 e4m3 stages of 128 latent columns.
-      if (lane == 0) {
+      // ---- TMA producer warp (one lane issues).  BF16 cache: 9 query
+      // stages per piece, then 9 per 2-page block.  FP8 cache: 8 query
+      // stages (latent columns) plus the query RoPE columns into their own
+      // buffer per piece, then per block one RoPE stage (bf16) and 4 e4m3
+      // stages of 128 latent columns.  A block's page ids are read one block
+      // ahead, so their load latency hides behind the previous block's
+      // stages.
+      {
+        const bool leader = elect_one();
         uint32_t zc = 0, pieces = 0;
         auto page_of = [&](int r, int j) {
           int page = p.block_table[size_t(r) * sv.max_pages + j];
@@ -460,31 +480,41 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         };
         auto stage = [&](uint32_t tx, uint32_t* dst) -> bool {
           const uint32_t s = zc % nz, ph = (zc / nz) & 1u;
-          if (!swait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
-          MLA_TR(0, 1, zc);
-          mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
+          if (!ewait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
+          if (leader) {
+            MLA_TR(0, 1, zc);
+            mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
+          }
           *dst = sbase + L::z + s * kZStage;
           return true;
         };
         each_piece(sv, [&](const Piece& pc) {
           const int r = pc.T / sv.tiles_per_req, qt = pc.T % sv.tiles_per_req;
           const int row0 = r * rows_total + qt * MLA_TILE_ROWS;
-          prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK,
-                           uint32_t(min(MLA_TILE_ROWS, p.q_rows - row0)) * MLA_D_QK * 2);
+          int npa = page_of(r, pc.p0), npb = pc.p0 + 1 < pc.p1 ? page_of(r, pc.p0 + 1) : 0;
+          if (leader)
+            prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK,
+                             uint32_t(min(MLA_TILE_ROWS, p.q_rows - row0)) * MLA_D_QK * 2);
           for (int c = 0; c < (kFp8 ? 8 : 9); ++c, ++zc) {
             uint32_t dst;
             if (!stage(kZStage, &dst)) return false;
             const uint32_t fb = bar(bars->z_full[zc % nz]);
-            tma_load_2d(dst, &q_map, 64 * c, row0, fb);
-            tma_load_2d(dst + kBox, &q_map, 64 * c, row0 + 64, fb);
+            if (leader) {
+              tma_load_2d(dst, &q_map, 64 * c, row0, fb);
+              tma_load_2d(dst + kBox, &q_map, 64 * c, row0 + 64, fb);
+            }
+            __syncwarp();
           }
           if constexpr (kFp8) {
             // the RoPE MMAs of the previous piece must be done with the buffer
-            if (!swait(ctl, bar(bars->qpe_empty), (pieces & 1u) ^ 1u)) return false;
+            if (!ewait(ctl, bar(bars->qpe_empty), (pieces & 1u) ^ 1u)) return false;
             const uint32_t fb = bar(bars->qpe_full);
-            mbar_arrive_expect_tx(fb, kZStage);
-            tma_load_2d(sbase + L::qpe, &q_map, MLA_D_V, row0, fb);
-            tma_load_2d(sbase + L::qpe + kBox, &q_map, MLA_D_V, row0 + 64, fb);
+            if (leader) {
+              mbar_arrive_expect_tx(fb, kZStage);
+              tma_load_2d(sbase + L::qpe, &q_map, MLA_D_V, row0, fb);
+              tma_load_2d(sbase + L::qpe + kBox, &q_map, MLA_D_V, row0 + 64, fb);
+            }
+            __syncwarp();
           }
           ++pieces;
           for (int j = pc.p0; j < pc.p1; j += 2) {
@@ -493,33 +523,46 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               for (int u = 0; u < 2; ++u)
                 if (kPrefetchPages > 0 && j + u + kPrefetchPages < pc.p1) {
                   const int pg = page_of(r, j + u + kPrefetchPages);
-                  if (pg >= 0) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
+                  if (pg >= 0 && leader) prefetch_l2_bulk(p.kv + size_t(pg) * kPageBytes, kPageBytes);
                 }
             }
-            int pa = page_of(r, j), pb = two ? page_of(r, j + 1) : 0;
-            if (pa < 0 || pb < 0) flag_status(p.ws, kStatusBadPage);
+            int pa = npa, pb = two ? npb : 0;
+            if (j + 2 < pc.p1) {
+              npa = page_of(r, j + 2);
+              npb = j + 3 < pc.p1 ? page_of(r, j + 3) : 0;
+            }
+            if ((pa < 0 || pb < 0) && leader) flag_status(p.ws, kStatusBadPage);
             pa = max(pa, 0);     // any valid page; the consumers mask every token of it
             pb = max(pb, 0);
             if constexpr (kFp8) {
               uint32_t dst;
               if (!stage(two ? kZStage : kBox, &dst)) return false;
               uint32_t fb = bar(bars->z_full[zc % nz]);
-              tma_load_3d(dst, &rope_map, 0, 0, pa, fb);
-              if (two) tma_load_3d(dst + kBox, &rope_map, 0, 0, pb, fb);
+              if (leader) {
+                tma_load_3d(dst, &rope_map, 0, 0, pa, fb);
+                if (two) tma_load_3d(dst + kBox, &rope_map, 0, 0, pb, fb);
+              }
+              __syncwarp();
               ++zc;
               for (int c = 0; c < 4; ++c, ++zc) {
                 if (!stage(two ? kZStage : kBox, &dst)) return false;
                 fb = bar(bars->z_full[zc % nz]);
-                tma_load_3d(dst, &pool_map, 128 * c, 0, pa, fb);
-                if (two) tma_load_3d(dst + kBox, &pool_map, 128 * c, 0, pb, fb);
+                if (leader) {
+                  tma_load_3d(dst, &pool_map, 128 * c, 0, pa, fb);
+                  if (two) tma_load_3d(dst + kBox, &pool_map, 128 * c, 0, pb, fb);
+                }
+                __syncwarp();
               }
             } else {
               for (int c = 0; c < 9; ++c, ++zc) {
                 uint32_t dst;
                 if (!stage(two ? kZStage : kBox, &dst)) return false;
                 const uint32_t fb = bar(bars->z_full[zc % nz]);
-                tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
-                if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
+                if (leader) {
+                  tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
+                  if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
+                }
+                __syncwarp();
               }
             }
           }
@@ -1112,12 +1155,12 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           drain_wait(bar(bars->v_loaded[idx % NV]), (idx / NV) & 1u);
         }
       }
-    } else if (warp >= 8) {
+    } else if (conv_rank(warp) >= 0) {
       // ---- V converters: each landed stage is rewritten in place from bf16
       // to fp16 (same size, same swizzled N-major layout).  Tokens at or
       // past the request's length become zero: their bytes may be anything
       // and 0 * NaN would poison O.  Thread -> 16 chunks of 16 bytes.
-      const int ct = tid - 256;
+      const int ct = conv_rank(warp) * 32 + lane;
       uint32_t vc = 0;
       each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req;
