@@ -54,8 +54,14 @@ namespace {
 
 using namespace ptx;
 
-constexpr int NZ = 11;  // 16 KB stages of the score CTA's ring (bf16 cache)
-constexpr int NZ8 = 6;  // the same ring for the FP8 cache (e4m3 and RoPE stages)
+// Score CTA ring.  BF16 cache: 5 stages of 32 KB, each two 64-column boxes
+// of both pages (the ninth box, the RoPE columns, alone in the fifth), so
+// the QK issuer waits once per 8 MMAs: each wait in the issuing thread idles
+// the tensor pipe, whose queue holds only a few MMAs.  FP8 cache: 6 stages
+// of 16 KB (e4m3 and RoPE stages).
+constexpr int NZ = 5;
+constexpr int NZ8 = 6;
+constexpr int kNZMax = 6;
 constexpr int NC = 4;   // FP8 cache: 16 KB stages of fp16 cache rows converted from e4m3
 // P page slots (output CTA): slot 0 takes page 0 of a block with the block's
 // rescale factors and row sums, slot 1 its page 1.  Each is refilled as soon
@@ -95,7 +101,7 @@ constexpr uint32_t kTmemSLat = 256;                   // FP8 cache: latent-part 
 
 struct Bars {
   // score CTA (FP8 cache: also the converted ring and the query RoPE buffer)
-  uint64_t z_full[NZ], z_empty[NZ], s_full, s_empty, q_ready, x_free[NX];
+  uint64_t z_full[kNZMax], z_empty[kNZMax], s_full, s_empty, q_ready, x_free[NX];
   uint64_t c_full[NC], c_empty[NC], qpe_full, qpe_empty;
   // output CTA
   uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_go, corr_done, pv_blk[NB], o_free;
@@ -117,8 +123,9 @@ constexpr uint32_t kOffData = 1024;
 template <bool kFp8>
 struct LayS {
   static constexpr int nz = kFp8 ? NZ8 : NZ;
+  static constexpr uint32_t zbytes = kFp8 ? kZStage : 2 * kZStage;   // bytes per ring stage
   static constexpr uint32_t z = kOffData;
-  static constexpr uint32_t c = z + nz * kZStage;
+  static constexpr uint32_t c = z + nz * zbytes;
   static constexpr uint32_t qpe = c + (kFp8 ? NC * kZStage : 0u);
   static constexpr uint32_t stage = qpe + (kFp8 ? kZStage : 0u);
   static constexpr uint32_t xchg = stage + kPStage;               // row max / sum exchange
@@ -400,7 +407,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   if (tid == 0) {
     // FP8 cache: a ring stage is refilled once the softmax, the issuer and
     // the converters have each released it (see the issuer)
-    for (int s = 0; s < NZ; ++s) {
+    for (int s = 0; s < kNZMax; ++s) {
       mbar_init(bar(bars->z_full[s]), 1);
       mbar_init(bar(bars->z_empty[s]), kFp8 ? 3 : 1);
     }
@@ -485,7 +492,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             MLA_TR(0, 1, zc);
             mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
           }
-          *dst = sbase + L::z + s * kZStage;
+          *dst = sbase + L::z + s * L::zbytes;
           return true;
         };
         each_piece(sv, [&](const Piece& pc) {
@@ -495,13 +502,20 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           if (leader)
             prefetch_l2_bulk(p.q + size_t(row0) * MLA_D_QK,
                              uint32_t(min(MLA_TILE_ROWS, p.q_rows - row0)) * MLA_D_QK * 2);
-          for (int c = 0; c < (kFp8 ? 8 : 9); ++c, ++zc) {
+          // query boxes: FP8 cache one per stage (8), BF16 cache two per
+          // stage (9 in 5 stages)
+          constexpr int nqs = kFp8 ? 8 : 5, qbs = kFp8 ? 1 : 2;
+          for (int q = 0; q < nqs; ++q, ++zc) {
+            const int nb = kFp8 ? 1 : (q < 4 ? 2 : 1);
             uint32_t dst;
-            if (!stage(kZStage, &dst)) return false;
+            if (!stage(uint32_t(nb) * kZStage, &dst)) return false;
             const uint32_t fb = bar(bars->z_full[zc % nz]);
             if (leader) {
-              tma_load_2d(dst, &q_map, 64 * c, row0, fb);
-              tma_load_2d(dst + kBox, &q_map, 64 * c, row0 + 64, fb);
+              for (int k = 0; k < nb; ++k) {
+                const int c = qbs * q + k;
+                tma_load_2d(dst + uint32_t(k) * kZStage, &q_map, 64 * c, row0, fb);
+                tma_load_2d(dst + uint32_t(k) * kZStage + kBox, &q_map, 64 * c, row0 + 64, fb);
+              }
             }
             __syncwarp();
           }
@@ -554,13 +568,18 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                 __syncwarp();
               }
             } else {
-              for (int c = 0; c < 9; ++c, ++zc) {
+              // stage q: boxes 2q and 2q + 1 (box 8 alone), each both pages
+              for (int q = 0; q < 5; ++q, ++zc) {
+                const int nb = q < 4 ? 2 : 1;
                 uint32_t dst;
-                if (!stage(two ? kZStage : kBox, &dst)) return false;
+                if (!stage(uint32_t(nb) * (two ? kZStage : kBox), &dst)) return false;
                 const uint32_t fb = bar(bars->z_full[zc % nz]);
                 if (leader) {
-                  tma_load_3d(dst, &pool_map, 64 * c, 0, pa, fb);
-                  if (two) tma_load_3d(dst + kBox, &pool_map, 64 * c, 0, pb, fb);
+                  for (int k = 0; k < nb; ++k) {
+                    const int c = 2 * q + k;
+                    tma_load_3d(dst + uint32_t(k) * kZStage, &pool_map, 64 * c, 0, pa, fb);
+                    if (two) tma_load_3d(dst + uint32_t(k) * kZStage + kBox, &pool_map, 64 * c, 0, pb, fb);
+                  }
                 }
                 __syncwarp();
               }
@@ -577,8 +596,8 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         if (kFp8 && pieces > 0) drain_wait(bar(bars->qpe_full), (pieces - 1) & 1u);
       }
     } else if (warp == 1) {
-      // ---- QK^T issuer warp: per block 36 MMAs M128 N128 K16.  BF16 cache: 9
-      // stages x 4, A = Q (TMEM), into S.  FP8 cache: the RoPE stage x 4 with
+      // ---- QK^T issuer warp: per block 36 MMAs M128 N128 K16.  BF16 cache: 5
+      // stages of 2 boxes (the last 1) x 4 MMAs, A = Q (TMEM), into S.  FP8 cache: the RoPE stage x 4 with
       // A = the query RoPE columns (shared memory) into S_rope, then 8
       // converted fp16 stages x 4 with A = the fp16 query (TMEM) into S_lat.
       // The warp waits and computes operands together; one lane issues.
@@ -595,7 +614,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         // after three releases: softmax, issuer, converter.  For the RoPE
         // and e4m3 stages, which the softmax never sees, the issuer releases
         // twice.
-        constexpr int nq = kFp8 ? 8 : 9;
+        constexpr int nq = kFp8 ? 8 : 5;   // ring stages of the query
         if constexpr (kFp8) {
           for (int u = 0; u < nq; ++u, ++zc) {
             if (!ewait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
@@ -658,18 +677,25 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               __syncwarp();
             }
           } else {
-            for (int c = 0; c < 9; ++c, ++zc) {
+            for (int q = 0; q < 5; ++q, ++zc) {
               const uint32_t zs = zc % nz;
               if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-              if (leader) MLA_TR(1, 10 + c, bc);
+              if (leader) MLA_TR(1, 10 + q, bc);
               tc_fence_after();
-              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
-              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemS;
+              const uint32_t d = tmem + kTmemS;
               if (leader) {
-                mma_ts(d, ad, bd, kIdescQK, c != 0);
-                mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
-                mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
-                mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                  const int c = 2 * q + k;
+                  if (c < 9) {
+                    const uint64_t bd = zdesc0 + uint64_t((zs * L::zbytes + uint32_t(k) * kZStage) >> 4);
+                    const uint32_t ad = tmem + 32u * uint32_t(c);
+                    mma_ts(d, ad, bd, kIdescQK, c != 0);
+                    mma_ts(d, ad + 8u, bd + 2u, kIdescQK, 1u);
+                    mma_ts(d, ad + 16u, bd + 4u, kIdescQK, 1u);
+                    mma_ts(d, ad + 24u, bd + 6u, kIdescQK, 1u);
+                  }
+                }
                 mma_commit(bar(bars->z_empty[zs]));
               }
               __syncwarp();
@@ -766,25 +792,27 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
         if (g == 0) MLA_TR(2, 9, bc);
-        // query row i -> TMEM lane i.  Box c of the query is stage zc + c
-        // (rows 0-63, then 64-127 at +8 KB).  BF16 cache: boxes 0-8 as bf16
-        // pairs in columns [0, 288), group 0 moves boxes 0-4, group 1 boxes
-        // 5-8.  FP8 cache: the latent boxes 0-7 as fp16 pairs in columns
-        // [0, 256) (the RoPE box stays in shared memory), 0-3 / 4-7.  Every QK
-        // MMA of the previous piece has completed: its last S was read.
+        // query row i -> TMEM lane i.  Box c of the query (rows 0-63, then
+        // 64-127 at +8 KB) is sub-stage c % qbs of stage zc + c / qbs.  BF16
+        // cache: boxes 0-8, two per stage, as bf16 pairs in columns [0, 288),
+        // group 0 moves boxes 0-4, group 1 boxes 5-8.  FP8 cache: the latent
+        // boxes 0-7, one per stage, as fp16 pairs in columns [0, 256) (the
+        // RoPE box stays in shared memory), 0-3 / 4-7.  Every QK MMA of the
+        // previous piece has completed: its last S was read.
         {
-          constexpr int nq = kFp8 ? 8 : 9, nq0 = kFp8 ? 4 : 5;
+          constexpr int nq = kFp8 ? 8 : 9, nq0 = kFp8 ? 4 : 5, qbs = kFp8 ? 1 : 2;
           const uint32_t roff = uint32_t(i >> 6) * kBox + uint32_t(i & 63) * 128;
           bool big = false;
 #pragma unroll 1
           for (int c = 0; c < nq; ++c) {
-            const uint32_t idx = zc + c;
-            if (!gwait(ctl, bar(bars->z_full[idx % nz]), (idx / nz) & 1u, g == 0, carry_ok)) return false;
+            const uint32_t idx = zc + uint32_t(c / qbs);
+            if (c % qbs == 0)
+              if (!gwait(ctl, bar(bars->z_full[idx % nz]), (idx / nz) & 1u, g == 0, carry_ok)) return false;
             // FP8 cache: every thread has passed the barrier, so the previous
             // query stage has been read: the producer may refill it
             if (kFp8 && c > 0 && g == 0) mbar_arrive(bar(bars->z_empty[(idx - 1) % nz]));
             if ((c < nq0) == (h == 0)) {
-              const uint32_t st = sbase + L::z + (idx % nz) * kZStage + roff;
+              const uint32_t st = sbase + L::z + (idx % nz) * L::zbytes + uint32_t(c % qbs) * kZStage + roff;
               uint32_t v[32];
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
@@ -806,7 +834,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             named_bar_sync(kSoftmaxBar, kSmThreads);
             if (g == 0) mbar_arrive(bar(bars->z_empty[(zc + nq - 1) % nz]));
           }
-          zc += nq + (kFp8 ? 5 : 9) * ((pc.p1 - pc.p0 + 1) / 2);
+          zc += (kFp8 ? 8u : 5u) + 5u * uint32_t((pc.p1 - pc.p0 + 1) / 2);   // query stages, then 5 per block
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
