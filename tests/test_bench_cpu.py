@@ -1,0 +1,56 @@
+"""bench.py on the host: its reference arm (the oracle timed on the CPU) runs
+and prints one well-formed JSON line, and every global name its functions use
+is defined (a broken bench must fail here, not on the GPU machine)."""
+import builtins
+import dis
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+import types
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _load_bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _loaded_globals(code):
+    """Names the code (and every function or lambda nested in it) loads as globals."""
+    names = {ins.argval for ins in dis.get_instructions(code) if ins.opname == "LOAD_GLOBAL"}
+    for c in code.co_consts:
+        if isinstance(c, types.CodeType):
+            names |= _loaded_globals(c)
+    return names
+
+
+def test_bench_functions_load_only_defined_globals():
+    b = _load_bench()
+    for name, obj in vars(b).items():
+        if isinstance(obj, types.FunctionType) and obj.__module__ == b.__name__:
+            undefined = sorted(n for n in _loaded_globals(obj.__code__)
+                               if n not in vars(b) and not hasattr(builtins, n))
+            assert not undefined, (name, undefined)
+    for fn in ("main", "run_ours", "run_reference", "run_e2e_pipelined"):
+        assert callable(getattr(b, fn, None)), fn
+
+
+def test_reference_arm_prints_its_json_line():
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
+         "--ref-requests", "1"],
+        cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = [l for l in out.stdout.splitlines() if l.startswith("{")][-1]
+    rec = json.loads(line)
+    assert rec["impl"] == "reference"
+    assert rec["value"] > 0 and rec["steps"] == 1 and rec["warmup"] == 0
+    assert rec["config"]["workload"] == "dsv3_b64_h128_t4096_paged"
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
+    assert rec["higher_is_better"] is True
