@@ -60,6 +60,33 @@ def test_split_counts_agree(n_sms):
     check_full(wl, n_sms=n_sms)
 
 
+def _growing_scores(name):
+    # A RoPE column equal to the token index (query column 1 there) makes the
+    # scores grow by softmax_scale * log2(e) ~ 0.10 log2 units per token: each
+    # 128-token block's max then exceeds the running max by ~13 > 8, so O is
+    # rescaled before nearly every block's PVs.
+    wl = mw.make(2, 1, 128, [4096, 1000], seed=12, name=name)
+    for r, t in enumerate(wl.seqlens):
+        for j in range((int(t) + 63) // 64):
+            page = int(wl.block_table[r, j])
+            wl.pool[page, :, 512] = torch.arange(64 * j, 64 * j + 64, dtype=torch.float32).to(torch.bfloat16)
+    wl.q[..., 512] = 1.0
+    return wl
+
+
+@pytest.mark.parametrize("n_sms", [None, 16])
+def test_running_max_rescales_every_block(n_sms):
+    # with 16 SMs also across split pieces, whose partials the combine merges
+    check_full(_growing_scores("rescale"), n_sms=n_sms)
+
+
+def test_fp8_running_max_rescales_every_block():
+    import dataclasses
+    wl = _growing_scores("rescale_fp8")
+    pool, ks = mw.quantize_fp8_pages(wl.pool)   # the RoPE part stays bf16
+    check_full(dataclasses.replace(wl, pool=pool, kv_scale=ks, cache_dtype="fp8"))
+
+
 def test_nan_in_unused_slots_and_pages():
     wl = mw.make(3, 1, 128, [70, 130, 1], seed=10, name="poison")
     O0, L0, _ = run(wl)
