@@ -95,7 +95,7 @@ constexpr int kConvThreads = 256;                     // output-CTA converter wa
 constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
 constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of the softmax warps
 constexpr uint32_t kConvBar = 2;                      // named barrier of a CTA's converter warps
-constexpr int kConvThreadsS = 128;                    // FP8 cache: score-CTA converters, warps 12..15
+constexpr int kConvThreadsS = 192;                    // FP8 cache: score-CTA converters, warps 2, 3, 12..15
 constexpr uint32_t kFp8PageBytes = 64 * 512 + 64 * 64 * 2;   // 64x512 e4m3, then 64x64 bf16 RoPE
 constexpr uint32_t kTmemSLat = 256;                   // FP8 cache: latent-part scores, columns 256..383
 
@@ -714,13 +714,16 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       if (leader) mma_commit(bar(bars->mma_done));
       __syncwarp();
       drain_wait(bar(bars->mma_done), 0);
-    } else if (kFp8 && warp >= 12) {
+    } else if (kFp8 && (warp == 2 || warp == 3 || warp >= 12)) {
       // ---- FP8 cache: converters.  Each e4m3 stage (128 latent columns of
       // the block's two pages) becomes two fp16 stages of 64 columns in the
       // K-major 128-byte-swizzled layout of the bf16 path.  e4m3 -> fp16 is
-      // exact.  Thread t owns token row t & 63 of page t >> 6.
-      const int t = tid - 384, pg = t >> 6, rr = t & 63;
-      const uint32_t sw = uint32_t(rr & 7);
+      // exact.  Six warps (2, 3 and 12-15): four left the stages' latency
+      // exposed.
+      const int t = (warp < 12 ? warp - 2 : warp - 10) * 32 + lane;
+      // chunk o (16 e4m3 values) is row o / 8 of the stage (page row / 64,
+      // token row % 64), 16-byte column o % 8; thread t takes o = t + 192u
+      constexpr int kCh = (128 * 8 + kConvThreadsS - 1) / kConvThreadsS;
       uint32_t zc = 0, cc = 0;
       // Thread 0 also walks the query and RoPE stages in order and releases
       // them (the converters' share of their three releases).
@@ -744,26 +747,33 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                    bwait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u);
             if (!named_bar_and(kConvBar, kConvThreadsS, ok)) return false;
             if (t == 0) MLA_TR(6, 1, zc);
-            const uint32_t src = sbase + L::z + zs * kZStage + uint32_t(pg) * kBox + uint32_t(rr) * 128;
-            uint4 in[8];
+            const uint32_t src = sbase + L::z + zs * kZStage;
+            uint4 in[kCh];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) in[k] = ld_shared_v4(src + ((uint32_t(k) ^ sw) << 4));
+            for (int u = 0; u < kCh; ++u) {
+              const int o = t + kConvThreadsS * u, r = o >> 3, k = o & 7;
+              if (o < 128 * 8)
+                in[u] = ld_shared_v4(src + uint32_t(r >> 6) * kBox + uint32_t(r & 63) * 128 +
+                                     ((uint32_t(k) ^ uint32_t(r & 7)) << 4));
+            }
             // every converter has read the stage: the producer may refill it
             named_bar_sync(kConvBar, kConvThreadsS);
             if (t == 0) mbar_arrive(bar(bars->z_empty[zs]));
-            const uint32_t row = uint32_t(pg) * kBox + uint32_t(rr) * 128;
-            const uint32_t d0 = sbase + L::c + c0 * kZStage + row, d1 = sbase + L::c + c1 * kZStage + row;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int u = 0; u < kCh; ++u) {
+              const int o = t + kConvThreadsS * u, r = o >> 3, k = o & 7;
+              if (o >= 128 * 8) continue;
               // 16 e4m3 values (latent columns 16k..16k+15 of the box) -> fp16
               // chunks 2(k&3), 2(k&3)+1 of converted stage k >> 2
-              const uint32_t dst = (k < 4 ? d0 : d1);
+              const uint32_t sw = uint32_t(r & 7);
+              const uint32_t dst = sbase + L::c + (k < 4 ? c0 : c1) * kZStage + uint32_t(r >> 6) * kBox +
+                                   uint32_t(r & 63) * 128;
               const uint32_t ch = uint32_t(2 * (k & 3));
-              st_shared_v4(dst + ((ch ^ sw) << 4), e4m3x2_to_f16x2(in[k].x & 0xFFFFu), e4m3x2_to_f16x2(in[k].x >> 16),
-                           e4m3x2_to_f16x2(in[k].y & 0xFFFFu), e4m3x2_to_f16x2(in[k].y >> 16));
-              st_shared_v4(dst + (((ch + 1u) ^ sw) << 4), e4m3x2_to_f16x2(in[k].z & 0xFFFFu),
-                           e4m3x2_to_f16x2(in[k].z >> 16), e4m3x2_to_f16x2(in[k].w & 0xFFFFu),
-                           e4m3x2_to_f16x2(in[k].w >> 16));
+              st_shared_v4(dst + ((ch ^ sw) << 4), e4m3x2_to_f16x2(in[u].x & 0xFFFFu), e4m3x2_to_f16x2(in[u].x >> 16),
+                           e4m3x2_to_f16x2(in[u].y & 0xFFFFu), e4m3x2_to_f16x2(in[u].y >> 16));
+              st_shared_v4(dst + (((ch + 1u) ^ sw) << 4), e4m3x2_to_f16x2(in[u].z & 0xFFFFu),
+                           e4m3x2_to_f16x2(in[u].z >> 16), e4m3x2_to_f16x2(in[u].w & 0xFFFFu),
+                           e4m3x2_to_f16x2(in[u].w >> 16));
             }
             fence_proxy_async_cta();   // the stages feed the tensor core
             mbar_arrive(bar(bars->c_full[c0]));
