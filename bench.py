@@ -206,9 +206,12 @@ def run_reference(args, wl, world, rank):
 
 def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
     """Steps per unit time of the whole decode step including its host
-    transfers, pipelined over three streams (upload, compute, download)."""
+    transfers, pipelined over three streams (upload, compute, download).
+    With three buffer sets a step's upload never waits for the download of
+    the step before last, so uploads and downloads each run back to back on
+    their own copy engine."""
     import mla_latent_space_b200 as mla
-    nbuf = 2
+    nbuf = args.e2e_buffers
     h_q = wl.q.pin_memory()
     h_bt = torch.from_numpy(wl.block_table).pin_memory()
     h_sl = torch.from_numpy(wl.seqlens).pin_memory()
@@ -251,8 +254,15 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
             down_done[b].record(s_down)
         used[b] = True
 
-    for k in range(max(3, args.warmup)):
+    # warm-up: the host link only reaches its full rate after some hundreds of
+    # milliseconds of steady transfers (cold, an upload runs at a quarter of
+    # it), as it would in a serving loop; run steps for at least 0.3 s
+    k, t_warm = 0, time.perf_counter()
+    while k < max(3, args.warmup) or time.perf_counter() - t_warm < 0.3:
         step(k)
+        k += 1
+        if k % 64 == 0:
+            torch.cuda.synchronize()
     torch.cuda.synchronize()
     for dd in decs:
         st = dd.status()
@@ -389,7 +399,7 @@ def run_ours(args, wl, world, rank, local):
             "clocks": clk,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                    "pipelining": "upload / compute / download streams, 2 buffers"},
+                    "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers"},
             "gpu_launches": 3 * K}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10 s of oracle work: the sample repeated until 10 s have passed
@@ -413,6 +423,7 @@ def main():
     ap.add_argument("--config", type=int, default=2, help="workload 1-5 (2 = the headline decode batch)")
     ap.add_argument("--simt", action="store_true", help="time the SIMT debug kernel instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
     ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per decode launch for the current kernel (else null)")
