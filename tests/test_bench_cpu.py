@@ -54,3 +54,54 @@ def test_reference_arm_prints_its_json_line():
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
     assert rec["higher_is_better"] is True
+
+
+def _free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    # two ranks on gloo: rank 0 alone times the oracle and prints the line,
+    # rank 1 exits without work; both exit 0
+    out = subprocess.run(
+        [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+         "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+         os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+         "--ref-requests", "1"],
+        cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+
+
+def _ranks_body(rank, port, results):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE="2", RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    b = _load_bench()
+    world, r, _ = b.dist_setup(2)
+    try:
+        b.barrier(world)
+        results[r] = b.max_over_ranks(float(10 * r + 1), world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_barrier_and_max_over_ranks_on_gloo():
+    import torch.multiprocessing as mp
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        ctx = mp.get_context("spawn")
+        ps = [ctx.Process(target=_ranks_body, args=(r, port, results)) for r in range(2)]
+        for p in ps:
+            p.start()
+        for p in ps:
+            p.join(300)
+        assert all(p.exitcode == 0 for p in ps)
+        assert dict(results) == {0: 11.0, 1: 11.0}
