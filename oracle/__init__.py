@@ -4,5 +4,5 @@ Test infrastructure: only the tests, ``__graft_entry__.smoke()`` and the CPU
 baseline legs of ``bench.py`` may import it.  It shares no code with the
 CUDA path (``mla_latent_space_b200``) and never imports it.
 """
-from .mla_decode import (attend, brute, bf16_to_f64, combine, decode, decode_chunk,  # noqa: F401
-                         e4m3_table, gather_rows, page_rows_f64, round_bf16, visible_len)
+from .mla_decode import (absorb, attend, brute, bf16_to_f64, combine, decode, decode_chunk,  # noqa: F401
+                         decompress, e4m3_table, gather_rows, page_rows_f64, round_bf16, visible_len)

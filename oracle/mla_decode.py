@@ -26,6 +26,18 @@ plain definition, written out per (request, query token), in float64:
   5. O[r, i, h, c] = sum_j exp(x_j - lse) * C_j[c], c < 512.
 
 L <= 0 gives O = 0 and lse = -inf.
+
+The two per-head projections on either side of that attention (same page,
+"Absorption Trick": the key up-projection is folded into the query, and the
+output of the latent attention is decompressed by a separate GEMM) are
+written out as their definitions too, with d = 128 head dims and p = 64 RoPE
+dims:
+
+  absorb:      Qz[.., j, c] = sum_n q[.., j, n] * Wk[j, c, n]   (c < 512, n < d)
+               Qz[.., j, 512 + e] = q[.., j, d + e]             (e < p)
+               -- q = [q_nope | q_pe]; head j's keys are K_j = Z . Wk_j
+               (Wk_j is 512 x d), so Q . K_j^T = (Q . Wk_j^T) . Z^T.
+  decompress:  out[.., j, v] = sum_c O[.., j, c] * Wkvb2[j, v, c]  (v < d)
 """
 from __future__ import annotations
 
@@ -37,6 +49,8 @@ import torch
 PAGE = 64
 D_QK = 576
 D_V = 512
+D_HEAD = 128
+D_ROPE = 64
 
 
 # ----------------------------------------------------------------------------
@@ -225,3 +239,28 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
         r = np.round(x / ulp) * ulp                  # np.round: ties to even
         r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, x), r)
     return np.where(np.isfinite(x), r, x)
+
+
+# ----------------------------------------------------------------------------
+# projections on either side of the latent attention
+# ----------------------------------------------------------------------------
+
+def absorb(q: np.ndarray, w_k: np.ndarray) -> np.ndarray:
+    """Absorbed query rows (page "MLA Cost Analysis & Regime Guide",
+    "Absorption Trick": Q . K^T = (Q . Wk^T) . Z^T).
+
+    q    float64 [..., h, d + p] = [q_nope | q_pe]
+    w_k  float64 [h, 512, d]: head j's keys are K_j = Z . w_k[j]
+    Returns float64 [..., h, 576] = [q_nope . w_k[j]^T | q_pe]."""
+    lat = np.einsum("...jn,jcn->...jc", q[..., :D_HEAD], w_k)
+    return np.concatenate([lat, q[..., D_HEAD:D_HEAD + D_ROPE]], axis=-1)
+
+
+def decompress(o_lat: np.ndarray, w_kvb2: np.ndarray) -> np.ndarray:
+    """Per-head output of the latent attention mapped back to head space
+    (same page and section: O_latent . W_kvb2^T, run after the attention).
+
+    o_lat   float64 [..., h, 512]
+    w_kvb2  float64 [h, d, 512]: head j's values are V_j = Z . w_kvb2[j]^T
+    Returns float64 [..., h, d]."""
+    return np.einsum("...jc,jvc->...jv", o_lat, w_kvb2)

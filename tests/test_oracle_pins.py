@@ -178,6 +178,49 @@ def test_absorption_identity():
     assert np.max(np.abs(got - ref)) < 1e-12
 
 
+def test_absorb_and_decompress_reach_plain_mha():
+    # the oracle's projections around its attention give the same heads as
+    # ordinary MHA over decompressed keys and values: q = [q_nope | q_pe],
+    # Wk_h is 512 x d (K_h = Z Wk_h), W_kvb2_h = Wv_h^T is d x 512
+    Wk, Wv, qn, qp, Z, KPE = case = _absorption_case(seed=3, t=130, h=5)
+    ref = _mha_reference(*case).numpy()
+    q = torch.cat([qn, qp], dim=1).numpy()                       # h, 192
+    qz = oracle.absorb(q, Wk.numpy())                            # h, 576
+    C = torch.cat([Z, KPE], dim=1).numpy()
+    olat, _ = oracle.attend(qz, C, SCALE)
+    got = oracle.decompress(olat, Wv.transpose(1, 2).numpy())
+    assert got.shape == ref.shape == (5, 128)
+    assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_projections_on_selector_weights():
+    # closed forms: a weight that selects one input column per output column,
+    # scaled differently per head, must route exactly those values
+    g = torch.Generator().manual_seed(11)
+    R, h = 3, 4
+    q = torch.randn(R, h, 192, generator=g, dtype=torch.float64).numpy()
+    wk = np.zeros((h, 512, 128))
+    for j in range(h):
+        for n in range(128):
+            wk[j, (n + 100 * j) % 512, n] = j + 1.0              # latent c <- (j+1) q_nope[n]
+    qz = oracle.absorb(q, wk)
+    want = np.zeros((R, h, 576))
+    for j in range(h):
+        for n in range(128):
+            want[:, j, (n + 100 * j) % 512] = (j + 1.0) * q[:, j, n]
+    want[..., 512:] = q[..., 128:]
+    assert np.array_equal(qz, want)
+    o = torch.randn(R, h, 512, generator=g, dtype=torch.float64).numpy()
+    wv = np.zeros((h, 128, 512))
+    for j in range(h):
+        for v in range(128):
+            wv[j, v, (3 * v + 128 * j) % 512] = -(j + 2.0)
+    out = oracle.decompress(o, wv)
+    for j in range(h):
+        for v in range(128):
+            assert np.array_equal(out[:, j, v], -(j + 2.0) * o[:, j, (3 * v + 128 * j) % 512])
+
+
 def test_uniform_scores_give_mean_of_values():
     # Q = 0: every score is 0, so the weights are 1/L, O is the mean of the
     # value rows and lse = ln L
