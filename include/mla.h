@@ -61,6 +61,8 @@ enum {
 #define MLA_D_V 512
 #define MLA_PAGE_SIZE 64
 #define MLA_TILE_ROWS 128
+#define MLA_D_HEAD 128 /* d: per-head query/key/value dims before absorption */
+#define MLA_D_ROPE 64  /* p: RoPE dims (the last 64 of the 576)              */
 
 /* Problem description.  Every field is read on the host only. */
 typedef struct {
@@ -190,6 +192,36 @@ int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, const void* 
                            const float* kv_scale, const int32_t* block_table,
                            const int32_t* seqlens, float softmax_scale, void* out, float* lse,
                            int32_t* device_status, void* stream);
+
+/* ---- the projections on either side of the decode -------------------------
+ * "MLA Cost Analysis & Regime Guide", section "Absorption Trick": the key
+ * up-projection Wk is folded into the query (Q . K^T = (Q . Wk^T) . Z^T),
+ * and the latent output is decompressed by a separate GEMM after the
+ * attention (O_latent . W_kvb2^T).  Both run on the tensor core (tcgen05,
+ * bf16 operands, fp32 accumulation, bf16 result rounded to nearest even).
+ * rows = batch * s_q query rows; every tensor is dense row-major and its
+ * pointer 16-byte aligned; inputs and outputs must not overlap.  rows == 0
+ * enqueues nothing and returns MLA_OK (pointers unchecked).  device_status: optional device int32 (4-byte aligned)
+ * that a bounded wait which gave up ORs 1 into (NULL to skip; never cleared
+ * by these calls).  Returns MLA_OK, MLA_ERR_INVALID_ARG (null or misaligned
+ * pointer, rows < 0, num_heads outside [1, 65535]) or MLA_ERR_CUDA. */
+
+/* f1a -- absorbed query rows, the q argument of mla_decode_fwd:
+ *   qz[r, j, c]       = sum_n q[r, j, n] * w_k[j, c, n]   (c < 512, n < 128)
+ *   qz[r, j, 512 + e] = q[r, j, 128 + e]                  (e < 64, copied)
+ *   q   : bf16 [rows, num_heads, 192] = [q_nope 128 | q_pe 64] per head
+ *   w_k : bf16 [num_heads, 512, 128]; head j's keys are K_j = Z . w_k[j]
+ *   qz  : bf16 [rows, num_heads, 576] (written entirely) */
+int mla_absorb_q(int32_t rows, int32_t num_heads, const void* q, const void* w_k, void* qz,
+                 int32_t* device_status, void* stream);
+
+/* f1b -- output decompression of the latent attention result:
+ *   out[r, j, v] = sum_c o_lat[r, j, c] * w_kvb2[j, v, c]   (v < 128, c < 512)
+ *   o_lat  : bf16 [rows, num_heads, 512] (the out of mla_decode_fwd)
+ *   w_kvb2 : bf16 [num_heads, 128, 512]; head j's values are V_j = Z . w_kvb2[j]^T
+ *   out    : bf16 [rows, num_heads, 128] (written entirely) */
+int mla_decompress_o(int32_t rows, int32_t num_heads, const void* o_lat, const void* w_kvb2, void* out,
+                     int32_t* device_status, void* stream);
 
 /* Human-readable name of an MLA_* code (static storage). */
 const char* mla_error_string(int code);

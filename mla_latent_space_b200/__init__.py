@@ -22,6 +22,7 @@ MLA_OK = 0
 MLA_CACHE_BF16 = 0
 MLA_CACHE_FP8_E4M3 = 1
 D_QK, D_V, PAGE, TILE_ROWS = 576, 512, 64, 128
+D_HEAD, D_ROPE = 128, 64   # per-head dims before absorption, RoPE dims
 FP8_PAGE_BYTES = PAGE * D_V + PAGE * (D_QK - D_V) * 2
 
 EXPORTED = ("mla_schedule_bytes", "mla_workspace_bytes", "mla_get_schedule", "mla_decode_fwd",
@@ -71,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.mla_plan_schedule_host.restype = i32
         L.mla_decode_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
         L.mla_decode_fwd_noalloc.restype = i32
+        L.mla_absorb_q.argtypes = [i32, i32, vp, vp, vp, vp, vp]
+        L.mla_absorb_q.restype = i32
+        L.mla_decompress_o.argtypes = [i32, i32, vp, vp, vp, vp, vp]
+        L.mla_decompress_o.restype = i32
         L.mla_error_string.argtypes = [i32]
         L.mla_error_string.restype = ctypes.c_char_p
         L.mla_version.argtypes = []
@@ -223,6 +228,40 @@ def mla_get_device_status(sched, workspace, stream=None) -> int:
     _check(lib().mla_get_device_status(_ptr(sched), _ptr(workspace), _stream(stream), ctypes.byref(st)),
            "mla_get_device_status")
     return int(st.value)
+
+
+def _rows_heads(t: torch.Tensor, name: str, last: int):
+    if t.dim() < 2 or t.shape[-1] != last:
+        raise ValueError(f"{name} must have shape [..., heads, {last}], got {tuple(t.shape)}")
+    return t.numel() // (t.shape[-2] * last), t.shape[-2]
+
+
+def mla_absorb_q(q, w_k, qz, device_status: Optional[torch.Tensor] = None, stream=None):
+    """qz[..., j, :512] = q[..., j, :128] . w_k[j]^T and qz[..., j, 512:] =
+    q[..., j, 128:] on the tensor core.  q bf16 [..., h, 192], w_k bf16
+    [h, 512, 128], qz bf16 [..., h, 576] (the decode's query rows)."""
+    _need(q, "q", torch.bfloat16)
+    rows, h = _rows_heads(q, "q", D_HEAD + D_ROPE)
+    _need(w_k, "w_k", torch.bfloat16, (h, D_V, D_HEAD))
+    _need(qz, "qz", torch.bfloat16, tuple(q.shape[:-1]) + (D_QK,))
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32)
+    _check(lib().mla_absorb_q(int(rows), int(h), _ptr(q), _ptr(w_k), _ptr(qz), _ptr(device_status),
+                              _stream(stream)), "mla_absorb_q")
+
+
+def mla_decompress_o(o_lat, w_kvb2, out, device_status: Optional[torch.Tensor] = None, stream=None):
+    """out[..., j, v] = sum_c o_lat[..., j, c] w_kvb2[j, v, c] on the tensor
+    core.  o_lat bf16 [..., h, 512], w_kvb2 bf16 [h, 128, 512], out bf16
+    [..., h, 128]."""
+    _need(o_lat, "o_lat", torch.bfloat16)
+    rows, h = _rows_heads(o_lat, "o_lat", D_V)
+    _need(w_kvb2, "w_kvb2", torch.bfloat16, (h, D_HEAD, D_V))
+    _need(out, "out", torch.bfloat16, tuple(o_lat.shape[:-1]) + (D_HEAD,))
+    if device_status is not None:
+        _need(device_status, "device_status", torch.int32)
+    _check(lib().mla_decompress_o(int(rows), int(h), _ptr(o_lat), _ptr(w_kvb2), _ptr(out), _ptr(device_status),
+                                  _stream(stream)), "mla_decompress_o")
 
 
 class Decoder:

@@ -21,6 +21,10 @@ cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* 
 int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
                         const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
                         void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
+int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* qz, int32_t* status,
+                    cudaStream_t stream);
+int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
+                        cudaStream_t stream);
 }  // namespace mla
 
 using namespace mla;
@@ -192,6 +196,26 @@ int mla_get_device_status(const void* sched, void* workspace, void* stream, int*
   else if (all) *status = MLA_ERR_DEVICE_CHECK;
   else *status = MLA_OK;
   return MLA_OK;
+}
+
+int mla_absorb_q(int32_t rows, int32_t num_heads, const void* q, const void* w_k, void* qz, int32_t* device_status,
+                 void* stream) {
+  if (rows < 0 || num_heads < 1 || num_heads > 65535) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!q || !w_k || !qz) return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(w_k, 16) || !aligned(qz, 16) || !aligned(device_status, 4))
+    return MLA_ERR_INVALID_ARG;
+  return launch_absorb_q(rows, num_heads, q, w_k, qz, device_status, static_cast<cudaStream_t>(stream));
+}
+
+int mla_decompress_o(int32_t rows, int32_t num_heads, const void* o_lat, const void* w_kvb2, void* out,
+                     int32_t* device_status, void* stream) {
+  if (rows < 0 || num_heads < 1 || num_heads > 65535) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (!o_lat || !w_kvb2 || !out) return MLA_ERR_INVALID_ARG;
+  if (!aligned(o_lat, 16) || !aligned(w_kvb2, 16) || !aligned(out, 16) || !aligned(device_status, 4))
+    return MLA_ERR_INVALID_ARG;
+  return launch_decompress_o(rows, num_heads, o_lat, w_kvb2, out, device_status, static_cast<cudaStream_t>(stream));
 }
 
 const char* mla_error_string(int code) {

@@ -185,3 +185,35 @@ def config_shape(cfg: int, seed: int = 0):
     else:
         lens = np.full(kw["batch"], kw["seqlens"], dtype=np.int32)
     return kw["batch"], kw["s_q"], kw["num_heads"], lens
+
+
+D_HEAD = 128         # d: per-head query / key / value dims before absorption
+
+
+@dataclasses.dataclass
+class Projections:
+    """Inputs of the two per-head projections around the latent attention.
+
+    q       bf16 [rows, h, d + p]: [q_nope | q_pe] per head
+    w_k     bf16 [h, 512, d]: head j's keys are K_j = Z . w_k[j]
+    o_lat   bf16 [rows, h, 512]: latent attention output rows
+    w_kvb2  bf16 [h, d, 512]: head j's values are V_j = Z . w_kvb2[j]^T
+    """
+    q: torch.Tensor
+    w_k: torch.Tensor
+    o_lat: torch.Tensor
+    w_kvb2: torch.Tensor
+
+
+def make_projections(rows: int, num_heads: int, seed: int = 0) -> Projections:
+    """Draws, in this order from one generator: q ~ N(0, 1); w_k ~
+    N(0, 1/d) (so the absorbed latent query is about unit variance);
+    o_lat ~ N(0, 1); w_kvb2 ~ N(0, 1/512).  Every draw is rounded to bf16."""
+    gen = torch.Generator().manual_seed(seed)
+    h = num_heads
+    q = _randn_bf16(gen, (rows, h, D_HEAD + D_ROPE)) if rows else torch.empty((0, h, D_HEAD + D_ROPE),
+                                                                               dtype=torch.bfloat16)
+    w_k = (torch.randn((h, D_V, D_HEAD), generator=gen) / math.sqrt(D_HEAD)).to(torch.bfloat16)
+    o_lat = _randn_bf16(gen, (rows, h, D_V)) if rows else torch.empty((0, h, D_V), dtype=torch.bfloat16)
+    w_kvb2 = (torch.randn((h, D_HEAD, D_V), generator=gen) / math.sqrt(D_V)).to(torch.bfloat16)
+    return Projections(q, w_k, o_lat, w_kvb2)

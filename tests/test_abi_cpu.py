@@ -104,6 +104,23 @@ def test_schedule_and_combine_reject_bad_args():
     assert L.mla_get_device_status(None, fake, None, None) == -1
 
 
+def test_projections_reject_bad_args_before_any_launch():
+    L = mla.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    for fn in (L.mla_absorb_q, L.mla_decompress_o):
+        assert fn(4, 128, None, fake, fake, None, None) == -1
+        assert fn(4, 128, fake, None, fake, None, None) == -1
+        assert fn(4, 128, fake, fake, None, None, None) == -1
+        assert fn(-1, 128, fake, fake, fake, None, None) == -1
+        assert fn(4, 0, fake, fake, fake, None, None) == -1
+        assert fn(4, 65536, fake, fake, fake, None, None) == -1
+        assert fn(4, 128, odd, fake, fake, None, None) == -1                 # 16-byte alignment
+        assert fn(4, 128, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), None) == -1
+        assert fn(0, 128, fake, fake, fake, None, None) == 0                 # nothing to do, nothing enqueued
+        assert fn(0, 128, None, None, None, None, None) == 0
+
+
 # --------------------------------------------------------------------------
 # host scheduler
 # --------------------------------------------------------------------------
