@@ -286,6 +286,87 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
     return max_over_ranks(t0.elapsed_time(t1) / K, world)
 
 
+def proj_bytes(rows, heads):
+    """Algorithmic bytes of the two projections (weights read once, inputs
+    read once, outputs written once; bf16)."""
+    absorb = 2 * (heads * 512 * 128 + rows * heads * 192 + rows * heads * 576)
+    decompress = 2 * (heads * 128 * 512 + rows * heads * 512 + rows * heads * 128)
+    return absorb, decompress
+
+
+def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
+    """The per-head projections on either side of the latent decode, timed
+    like the decode (L2 flushed before each launch, CUDA events on the
+    launching stream), and the whole MLA decode attention they form with it:
+    absorb -> schedule -> decode -> combine -> decompress."""
+    import mla_latent_space_b200 as mla
+    R, h = wl.batch * wl.s_q, wl.num_heads
+    p = mw.make_projections(R, h, seed=1)
+    q = p.q.to(dev).view(wl.batch, wl.s_q, h, 192)
+    wk, wv = p.w_k.to(dev), p.w_kvb2.to(dev)
+    o_lat = p.o_lat.to(dev).view(wl.batch, wl.s_q, h, 512)
+    qz = torch.empty((wl.batch, wl.s_q, h, 576), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((wl.batch, wl.s_q, h, 128), dtype=torch.bfloat16, device=dev)
+    lat = torch.empty((wl.batch, wl.s_q, h, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.s_q, h), dtype=torch.float32, device=dev)
+    dec = mla.Decoder(shape, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def absorb():
+        mla.mla_absorb_q(q, wk, qz, device_status=status)
+
+    def decompress():
+        mla.mla_decompress_o(o_lat, wv, out, device_status=status)
+
+    def chain():
+        mla.mla_absorb_q(q, wk, qz, device_status=status)
+        dec.schedule(sl)
+        dec.decode(qz, pool, kv_scale, bt, sl, wl.softmax_scale, lat, lse)
+        mla.mla_decompress_o(lat, wv, out, device_status=status)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / len(evs) * 1e3   # us
+
+    # calibration: a one-element torch kernel timed in the same position
+    # (after the flush, between an event pair) shows what the event pair
+    # itself adds to a short launch
+    tiny = torch.zeros(1024, device=dev)
+    empty_us = timed(lambda: tiny.add_(1.0))
+    ab, db = proj_bytes(R, h)
+    res = {"empty_launch_us": empty_us}
+    for name, fn, by, kern in [("absorb", absorb, ab, "mla_absorb_q"), ("decompress", decompress, db, "mla_decompress_o")]:
+        us = timed(fn)
+        gbs = by / (us * 1e-6) / 1e9
+        net = max(us - empty_us, 1e-3)
+        res[name] = {"kernel": kern, "launch_us": us, "bytes": by, "flops": 2 * R * h * 128 * 512,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / pk["hbm_gbs"],
+                                  "frac_net_of_empty_launch": by / (net * 1e-6) / 1e9 / pk["hbm_gbs"]}}
+    chain_us = timed(chain)
+    if int(status.item()) != 0 or dec.status() != 0:
+        raise RuntimeError("device status set in the projection timing")
+    flops, _ = cost.workload_cost(wl)
+    res["whole_step_us"] = chain_us
+    res["whole_step"] = "absorb -> schedule -> decode -> combine -> decompress, one event pair around it"
+    res["whole_step_tflops"] = (flops + 2 * 2 * R * h * 128 * 512) / (chain_us * 1e-6) / 1e12
+    res["rows"], res["heads"] = R, h
+    # timed launches: absorb alone, decompress alone, and the chain's five kernels
+    res["gpu_launches"] = args.steps * (1 + 1 + 5)
+    return res
+
+
 def run_ours(args, wl, world, rank, local):
     import mla_latent_space_b200 as mla
     from mla_latent_space_b200 import build
@@ -364,6 +445,8 @@ def run_ours(args, wl, world, rank, local):
     # wait for its upload; a buffer is reused only after the step that last
     # used it has been downloaded).  The cache (302 MB) is larger than L2.
     e2e_ms = run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world)
+    proj = None if args.no_projections else run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush,
+                                                              peaks()[0])
     h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
 
@@ -405,6 +488,8 @@ def run_ours(args, wl, world, rank, local):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers"},
             "gpu_launches": 3 * K}
+    if proj is not None:
+        line["mla_attention"] = proj
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10 s of oracle work: the sample repeated until 10 s have passed
         n_req = max(1, min(wl.batch, args.ref_requests))
@@ -427,6 +512,8 @@ def main():
     ap.add_argument("--config", type=int, default=2, help="workload 1-5 (2 = the headline decode batch)")
     ap.add_argument("--simt", action="store_true", help="time the SIMT debug kernel instead")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-projections", action="store_true",
+                    help="skip the timing of the query absorption / output decompression kernels")
     ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
     ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,

@@ -110,6 +110,14 @@ __device__ __forceinline__ void rope_store(const ProjArgs& a, int r, int head, c
   for (int k = 0; k < 8; ++k) dst[k] = v[k];
 }
 
+// 2-D tiled store from this CTA's shared memory (bulk group; elements
+// outside the tensor are not written).
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // Shared-memory descriptor of a K-major operand in 128-byte swizzle atoms
 // (8 rows x 128 bytes, atoms 1024 bytes apart).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
@@ -177,6 +185,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // launched as a programmatic dependent: the set-up above overlapped the
+  // previous kernel; its results are visible once this returns.  A kernel
+  // after this one may begin its own set-up now (it waits the same way).
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ---- TMA producer
@@ -370,9 +383,18 @@ int launch_proj(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& o
   a.n_tiles = (a.rows + kTileN - 1) / kTileN;
   const long long units = (long long)a.n_tiles * a.m_tiles * a.heads;
   if (units >= (1ll << 31)) return MLA_ERR_UNSUPPORTED;
-  const unsigned grid = unsigned(units < sms ? units : sms);
-  proj_sm100_kernel<KC><<<grid, kProjThreads, kProjSmem, stream>>>(w, x, o, a);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(units < sms ? units : sms));
+  cfg.blockDim = dim3(kProjThreads);
+  cfg.dynamicSmemBytes = kProjSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, proj_sm100_kernel<KC>, w, x, o, a);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace
