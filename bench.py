@@ -367,6 +367,25 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
     return res
 
 
+def run_projections_only(args, wl, world, rank):
+    """`--projections-only`: the projection timing of run_projections alone,
+    on this rank's GPU, printed as its own JSON line."""
+    import mla_latent_space_b200 as mla
+    from mla_latent_space_b200 import build
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages, wl.cache_dtype, wl.causal)
+    pool = wl.pool.to(dev)
+    kv_scale = None if wl.kv_scale is None else wl.kv_scale.to(dev)
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    sl = torch.from_numpy(wl.seqlens).to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    pk, _ = peaks()
+    res = run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk)
+    if rank == 0:
+        print(json.dumps({"workload": wl.name, "mla_attention": res}), flush=True)
+
+
 def run_ours(args, wl, world, rank, local):
     import mla_latent_space_b200 as mla
     from mla_latent_space_b200 import build
@@ -514,6 +533,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-projections", action="store_true",
                     help="skip the timing of the query absorption / output decompression kernels")
+    ap.add_argument("--projections-only", action="store_true",
+                    help="time only the query absorption / output decompression kernels and the whole step")
     ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
     ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,
@@ -524,6 +545,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, wl, world, rank)
+        elif args.projections_only:
+            run_projections_only(args, wl, world, rank)
         else:
             run_ours(args, wl, world, rank, local)
     finally:
