@@ -27,6 +27,13 @@ plain definition, written out per (request, query token), in float64:
 
 L <= 0 gives O = 0 and lse = -inf.
 
+Token-level sparse decode (the FlashMLA product page lists "token-level
+sparse attention" for decoding) takes, per query token (r, i), a list of
+cache positions instead of the dense prefix: the plain reading is the same
+softmax attention over exactly the listed rows, shared by all heads of that
+query token.  Positions outside [0, t_r) (-1 padding) are skipped; a position
+listed twice is two keys.
+
 The two per-head projections on either side of that attention (same page,
 "Absorption Trick": the key up-projection is folded into the query, and the
 output of the latent attention is decompressed by a separate GEMM) are
@@ -160,6 +167,25 @@ def decode(wl, rows=None):
         O[n], L[n] = attend(q, C, wl.softmax_scale)
     if rows is None:
         return O.reshape(b, s, h, D_V), L.reshape(b, s, h)
+    return O, L
+
+
+def sparse_decode(wl, indices: np.ndarray):
+    """Token-level sparse decode over the workload's cache.
+
+    indices: int [b, s, k] cache positions per query token; entries outside
+    [0, t_r) are skipped.  Returns (O float64 [b, s, h, 512], lse float64
+    [b, s, h])."""
+    b, s, h, _ = wl.q.shape
+    O = np.zeros((b, s, h, D_V))
+    L = np.zeros((b, s, h))
+    for r in range(b):
+        t = int(wl.seqlens[r])
+        C_all = gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale)
+        for i in range(s):
+            pos = [int(j) for j in indices[r, i] if 0 <= int(j) < t]
+            C = C_all[pos] if pos else np.zeros((0, D_QK))
+            O[r, i], L[r, i] = attend(bf16_to_f64(wl.q[r, i]), C, wl.softmax_scale)
     return O, L
 
 

@@ -221,6 +221,77 @@ def test_projections_on_selector_weights():
             assert np.array_equal(out[:, j, v], -(j + 2.0) * o[:, j, (3 * v + 128 * j) % 512])
 
 
+# ---- token-level sparse decode ---------------------------------------------
+
+def _rows_as_workload(wl, r, i, pos):
+    """A one-request workload whose contiguous cache holds exactly the bf16
+    rows at positions `pos` of request r, in that order, queried by (r, i)."""
+    n = len(pos)
+    pages = max(1, (n + 63) // 64)
+    pool = torch.zeros((pages, 64, 576), dtype=torch.bfloat16)
+    for k, j in enumerate(pos):
+        pool[k // 64, k % 64] = wl.pool[int(wl.block_table[r][j // 64]), j % 64]
+    return mw.Workload(name="rows", batch=1, s_q=1, num_heads=wl.num_heads, causal=False, cache_dtype="bf16",
+                       seqlens=np.array([n], dtype=np.int32),
+                       block_table=np.arange(pages, dtype=np.int32)[None, :], q=wl.q[r:r + 1, i:i + 1].clone(),
+                       pool=pool, kv_scale=None, softmax_scale=wl.softmax_scale)
+
+
+def test_sparse_with_every_position_is_the_dense_decode():
+    wl = _tiny([70, 130, 5], h=3, s_q=2)
+    idx = np.full((3, 2, 140), -1, dtype=np.int32)
+    for r, t in enumerate(wl.seqlens):
+        idx[r, :, :t] = np.arange(t)
+    O, L = oracle.sparse_decode(wl, idx)
+    Od, Ld = oracle.decode(wl)
+    assert np.max(np.abs(O - Od)) < 1e-12 and np.max(np.abs(L - Ld)) < 1e-12
+
+
+def test_sparse_matches_brute_force_on_the_selected_rows():
+    # the rows are found through the block table: a brute-force triple loop over
+    # a contiguous copy of exactly those rows must agree
+    wl = _tiny([150, 90], h=2, s_q=2, seed=8)
+    rng = np.random.default_rng(1)
+    idx = np.full((2, 2, 12), -1, dtype=np.int32)
+    for r, t in enumerate(wl.seqlens):
+        for i in range(2):
+            idx[r, i, :10] = rng.choice(int(t), size=10, replace=False)
+    idx[0, 1, 10] = 149          # the last position
+    idx[1, 0, 11] = 90           # one past the end: skipped
+    O, L = oracle.sparse_decode(wl, idx)
+    for r in range(2):
+        for i in range(2):
+            pos = [int(j) for j in idx[r, i] if 0 <= j < wl.seqlens[r]]
+            Ob, Lb = oracle.brute(_rows_as_workload(wl, r, i, pos))
+            assert np.max(np.abs(O[r, i] - Ob[0, 0])) < 1e-12
+            assert np.max(np.abs(L[r, i] - Lb[0, 0])) < 1e-12
+
+
+def test_sparse_order_padding_and_duplicates():
+    wl = _tiny([200], h=4, seed=9)
+    rng = np.random.default_rng(2)
+    sel = rng.choice(200, size=37, replace=False).astype(np.int32)
+    a = sel[None, None, :]
+    b = np.concatenate([rng.permutation(sel), [-1, -1, 200, 1000]]).astype(np.int32)[None, None, :]
+    Oa, La = oracle.sparse_decode(wl, a)
+    Ob, Lb = oracle.sparse_decode(wl, b)
+    assert np.max(np.abs(Oa - Ob)) < 1e-12 and np.max(np.abs(La - Lb)) < 1e-12     # order, padding
+    # a position listed twice is two keys: with keys {u, v} and u twice the
+    # weights are 2e^{x_u} : e^{x_v}
+    u, v = int(sel[0]), int(sel[1])
+    Od, Ld = oracle.sparse_decode(wl, np.array([[[u, v, u]]], dtype=np.int32))
+    C = om.gather_rows(wl.pool, wl.block_table, 0, 200)
+    q = om.bf16_to_f64(wl.q[0, 0])
+    xu, xv = SCALE * (q @ C[u]), SCALE * (q @ C[v])
+    wu = 2 * np.exp(xu) / (2 * np.exp(xu) + np.exp(xv))
+    want = wu[:, None] * C[u, :512] + (1 - wu)[:, None] * C[v, :512]
+    assert np.max(np.abs(Od[0, 0] - want)) < 1e-12
+    assert np.max(np.abs(Ld[0, 0] - np.log(2 * np.exp(xu) + np.exp(xv)))) < 1e-12
+    # nothing valid: O = 0, lse = -inf
+    Oz, Lz = oracle.sparse_decode(wl, np.array([[[-1, 200, -7]]], dtype=np.int32))
+    assert np.all(Oz == 0) and np.all(np.isneginf(Lz))
+
+
 def test_uniform_scores_give_mean_of_values():
     # Q = 0: every score is 0, so the weights are 1/L, O is the mean of the
     # value rows and lse = ln L
