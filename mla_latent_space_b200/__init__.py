@@ -72,6 +72,12 @@ def lib() -> ctypes.CDLL:
         L.mla_plan_schedule_host.restype = i32
         L.mla_decode_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, f32, vp, vp, vp, vp]
         L.mla_decode_fwd_noalloc.restype = i32
+        L.mla_sparse_workspace_bytes.argtypes = [sp, i32, i32]
+        L.mla_sparse_workspace_bytes.restype = sz
+        L.mla_sparse_decode_fwd.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp, sz, vp, vp, vp]
+        L.mla_sparse_decode_fwd.restype = i32
+        L.mla_sparse_get_device_status.argtypes = [sp, i32, i32, vp, vp, ctypes.POINTER(i32)]
+        L.mla_sparse_get_device_status.restype = i32
         L.mla_absorb_q.argtypes = [i32, i32, vp, vp, vp, vp, vp]
         L.mla_absorb_q.restype = i32
         L.mla_decompress_o.argtypes = [i32, i32, vp, vp, vp, vp, vp]
@@ -228,6 +234,40 @@ def mla_get_device_status(sched, workspace, stream=None) -> int:
     _check(lib().mla_get_device_status(_ptr(sched), _ptr(workspace), _stream(stream), ctypes.byref(st)),
            "mla_get_device_status")
     return int(st.value)
+
+
+def mla_sparse_workspace_bytes(shape: mla_shape_t, topk: int, n_sms: int) -> int:
+    return int(lib().mla_sparse_workspace_bytes(ctypes.byref(shape), int(topk), int(n_sms)))
+
+
+class SparseDecoder:
+    """Token-level sparse decode through the C ABI: holds the zero-filled
+    workspace (torch allocation) for one shape, list length and device."""
+
+    def __init__(self, shape: mla_shape_t, topk: int, device=None):
+        self.shape, self.topk = shape, int(topk)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.n_sms = num_sms(self.device)
+        nb = mla_sparse_workspace_bytes(shape, self.topk, self.n_sms)
+        if nb == 0:
+            raise MLAError(-2, "SparseDecoder: shape not supported (BF16 cache, causal=0, topk >= 1)")
+        self.workspace = torch.zeros(nb, dtype=torch.uint8, device=self.device)
+
+    def decode(self, q, kv_cache, block_table, seqlens, indices, softmax_scale, out, lse, stream=None):
+        sh = self.shape
+        _check_decode_tensors(sh, q, kv_cache, None, block_table, seqlens, out, lse)
+        _need(indices, "indices", torch.int32, (sh.batch, sh.s_q, self.topk))
+        rc = lib().mla_sparse_decode_fwd(ctypes.byref(sh), self.topk, _ptr(q), _ptr(kv_cache), _ptr(block_table),
+                                         _ptr(seqlens), _ptr(indices), float(softmax_scale), _ptr(self.workspace),
+                                         self.workspace.numel(), _ptr(out), _ptr(lse), _stream(stream))
+        _check(rc, "mla_sparse_decode_fwd")
+
+    def status(self, stream=None) -> int:
+        st = ctypes.c_int(0)
+        _check(lib().mla_sparse_get_device_status(ctypes.byref(self.shape), self.topk, self.n_sms,
+                                                  _ptr(self.workspace), _stream(stream), ctypes.byref(st)),
+               "mla_sparse_get_device_status")
+        return int(st.value)
 
 
 def _rows_heads(t: torch.Tensor, name: str, last: int):

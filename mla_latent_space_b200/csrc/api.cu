@@ -21,6 +21,10 @@ cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* 
 int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
                         const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
                         void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
+cudaError_t launch_sparse_gather(const int32_t* indices, int topk, const int32_t* seqlens, int batch, int s_q,
+                                 const int32_t* block_table, int max_pages, int num_pages, const void* pool,
+                                 void* scratch, int vpages, int32_t* vseqlens, int32_t* vbt, void* status_ws,
+                                 cudaStream_t stream);
 int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* qz, int32_t* status,
                     cudaStream_t stream);
 int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
@@ -101,6 +105,49 @@ int check_decode_args(const mla_shape_t* shape, const void* q, const void* kv, c
   if (!std::isfinite(scale)) return MLA_ERR_INVALID_ARG;
   if (cap_slots_for(ws_bytes) < 0) return MLA_ERR_WORKSPACE;
   return MLA_OK;
+}
+
+// Workspace of the sparse decode (every region 256-byte aligned): the
+// compacted lengths and identity block table of the b*s single-query
+// "virtual" requests, their schedule, the decode workspace, and the scratch
+// pages the selected rows are gathered into.
+struct SparseLayout {
+  mla_shape_t vshape;
+  int vpages;
+  size_t vseq, vbt, sched, sched_bytes, ws, ws_bytes, scratch, total;
+};
+
+bool sparse_layout(const mla_shape_t* s, int topk, int num_sms, SparseLayout* L) {
+  if (check_shape(s) != MLA_OK || topk < 1 || topk > (1 << 24) || num_sms < 1) return false;
+  if (s->cache_dtype != MLA_CACHE_BF16 || s->causal != 0) return false;
+  const int64_t V = int64_t(s->batch) * s->s_q;
+  const int64_t vpages = (topk + MLA_PAGE_SIZE - 1) / MLA_PAGE_SIZE;
+  if (V * vpages >= (int64_t(1) << 31)) return false;
+  mla_shape_t vs = *s;
+  vs.batch = int32_t(V);
+  vs.s_q = 1;
+  vs.max_pages_per_seq = int32_t(vpages);
+  vs.num_pages = int32_t(V * vpages);
+  vs.causal = 0;
+  if (check_shape(&vs) != MLA_OK) return false;
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  L->vshape = vs;
+  L->vpages = int(vpages);
+  size_t off = 0;
+  L->vseq = off;
+  off = up(off + 4 * size_t(V));
+  L->vbt = off;
+  off = up(off + 4 * size_t(V) * size_t(vpages));
+  L->sched = off;
+  L->sched_bytes = sched_bytes_for(&vs, num_sms);
+  off = up(off + L->sched_bytes);
+  L->ws = off;
+  L->ws_bytes = kStatusBytes + size_t(max_slots_for(num_workers_for(num_sms))) * kSlotBytes;
+  off = up(off + L->ws_bytes);
+  L->scratch = off;
+  off += size_t(V) * size_t(vpages) * MLA_PAGE_SIZE * (2 * MLA_D_QK);
+  L->total = off;
+  return true;
 }
 
 }  // namespace
@@ -196,6 +243,58 @@ int mla_get_device_status(const void* sched, void* workspace, void* stream, int*
   else if (all) *status = MLA_ERR_DEVICE_CHECK;
   else *status = MLA_OK;
   return MLA_OK;
+}
+
+size_t mla_sparse_workspace_bytes(const mla_shape_t* shape, int topk, int num_sms) {
+  SparseLayout L;
+  return sparse_layout(shape, topk, num_sms, &L) ? L.total : 0;
+}
+
+int mla_sparse_decode_fwd(const mla_shape_t* shape, int topk, const void* q, const void* kv_cache,
+                          const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
+                          float softmax_scale, void* workspace, size_t workspace_bytes, void* out, float* lse,
+                          void* stream) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  if (shape->cache_dtype != MLA_CACHE_BF16) return MLA_ERR_UNSUPPORTED;
+  if (shape->causal != 0 || topk < 1 || topk > (1 << 24)) return MLA_ERR_INVALID_ARG;
+  if (!q || !kv_cache || !block_table || !seqlens || !indices || !workspace || !out || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv_cache, 256) || !aligned(out, 16) || !aligned(lse, 4) ||
+      !aligned(block_table, 4) || !aligned(seqlens, 4) || !aligned(indices, 4) || !aligned(workspace, 256))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((rc = device_sms(&sms)) != MLA_OK) return rc;
+  SparseLayout L;
+  if (!sparse_layout(shape, topk, sms, &L)) return MLA_ERR_UNSUPPORTED;
+  if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(workspace);
+  int32_t* vseq = reinterpret_cast<int32_t*>(w + L.vseq);
+  int32_t* vbt = reinterpret_cast<int32_t*>(w + L.vbt);
+  void* sched = w + L.sched;
+  void* ws = w + L.ws;
+  void* scratch = w + L.scratch;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_sparse_gather(indices, topk, seqlens, shape->batch, shape->s_q, block_table, shape->max_pages_per_seq,
+                           shape->num_pages, kv_cache, scratch, L.vpages, vseq, vbt, ws, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const ShapeInfo si = shape_info(&L.vshape);
+  if (launch_schedule(vseq, si, num_workers_for(sms), static_cast<int32_t*>(sched), st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const int cap = cap_slots_for(L.ws_bytes);
+  rc = launch_decode_sm100(&L.vshape, q, scratch, nullptr, vbt, vseq, softmax_scale, sched, ws, cap, out, lse, st);
+  if (rc != MLA_OK) return rc;
+  return launch_combine(sched, ws, out, lse, si.batch * si.tiles_per_req, cap, st) == cudaSuccess ? MLA_OK
+                                                                                                  : MLA_ERR_CUDA;
+}
+
+int mla_sparse_get_device_status(const mla_shape_t* shape, int topk, int num_sms, void* workspace, void* stream,
+                                 int* status) {
+  SparseLayout L;
+  if (!workspace || !status || !sparse_layout(shape, topk, num_sms, &L)) return MLA_ERR_INVALID_ARG;
+  char* w = static_cast<char*>(workspace);
+  return mla_get_device_status(w + L.sched, w + L.ws, stream, status);
 }
 
 int mla_absorb_q(int32_t rows, int32_t num_heads, const void* q, const void* w_k, void* qz, int32_t* device_status,

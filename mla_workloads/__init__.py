@@ -217,3 +217,20 @@ def make_projections(rows: int, num_heads: int, seed: int = 0) -> Projections:
     o_lat = _randn_bf16(gen, (rows, h, D_V)) if rows else torch.empty((0, h, D_V), dtype=torch.bfloat16)
     w_kvb2 = (torch.randn((h, D_HEAD, D_V), generator=gen) / math.sqrt(D_V)).to(torch.bfloat16)
     return Projections(q, w_k, o_lat, w_kvb2)
+
+
+def make_sparse_indices(seqlens, s_q: int, topk: int, seed: int = 0, pad: int = 0) -> np.ndarray:
+    """Per query token, `topk - pad` distinct cache positions drawn uniformly
+    from the request's [0, t) (all of them, in random order, when t is
+    smaller), then -1 up to `topk`: int32 [b, s_q, topk].  Draws from one
+    generator, request by request, query token by query token."""
+    gen = torch.Generator().manual_seed(seed)
+    b = len(seqlens)
+    out = np.full((b, s_q, topk), -1, dtype=np.int32)
+    for r in range(b):
+        t = int(seqlens[r])
+        for i in range(s_q):
+            n = min(topk - pad, t)
+            if n > 0:
+                out[r, i, :n] = torch.randperm(t, generator=gen)[:n].numpy()
+    return out
