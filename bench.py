@@ -367,6 +367,59 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
     return res
 
 
+SPARSE_SHAPE = dict(batch=64, s_q=1, heads=128, seqlen=32768, topk=2048)
+
+
+def sparse_cost(b, s, h, topk):
+    """FLOPs and the fused-ideal bytes of a sparse decode: every listed row
+    read once (1152 B), Q read and O written once."""
+    flops = 2 * b * s * h * topk * (2 * 512 + 64)
+    nbytes = 2 * (b * s * h * 576 + b * s * h * 512) + b * s * topk * 1152
+    return flops, nbytes
+
+
+def run_sparse(args, dev, flush, pk):
+    """Token-level sparse decode on a DeepSeek-V3.2-style batch: 64 requests
+    of 32768 cached tokens, 2048 listed positions per query token, timed like
+    the decode (L2 flushed before each launch sequence, CUDA events)."""
+    import mla_latent_space_b200 as mla
+    S = SPARSE_SHAPE
+    wl = mw.make(S["batch"], S["s_q"], S["heads"], S["seqlen"], seed=40, name="sparse_b64_h128_t32768_k2048")
+    idx = mw.make_sparse_indices(wl.seqlens, S["s_q"], S["topk"], seed=41)
+    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages)
+    dec = mla.SparseDecoder(shape, S["topk"], device=dev)
+    q, pool = wl.q.to(dev), wl.pool.to(dev)
+    bt, sl = torch.from_numpy(wl.block_table).to(dev), torch.from_numpy(wl.seqlens).to(dev)
+    ix = torch.from_numpy(idx).to(dev)
+    out = torch.empty((wl.batch, wl.s_q, wl.num_heads, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.batch, wl.s_q, wl.num_heads), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        dec.decode(q, pool, bt, sl, ix, wl.softmax_scale, out, lse)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        dec.decode(q, pool, bt, sl, ix, wl.softmax_scale, out, lse)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if dec.status() != 0:
+        raise RuntimeError("device status set in the sparse decode timing")
+    us = sum(a.elapsed_time(b) for a, b in evs) / len(evs) * 1e3
+    flops, nbytes = sparse_cost(wl.batch, wl.s_q, wl.num_heads, S["topk"])
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del pool
+    return {"workload": wl.name, "topk": S["topk"], "us_per_call": us, "tflops": flops / (us * 1e-6) / 1e12,
+            "kernels": "gather -> schedule -> decode -> combine (4 launches)",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "bytes": nbytes,
+                         "note": "bytes of a fused design (each listed row read once); this composition moves "
+                                 "each row three times"},
+            "gpu_launches": 4 * args.steps}
+
+
 def run_projections_only(args, wl, world, rank):
     """`--projections-only`: the projection timing of run_projections alone,
     on this rank's GPU, printed as its own JSON line."""
@@ -381,9 +434,13 @@ def run_projections_only(args, wl, world, rank):
     sl = torch.from_numpy(wl.seqlens).to(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     pk, _ = peaks()
-    res = run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk)
+    if args.sparse_only:
+        res = {"sparse": run_sparse(args, dev, flush, pk)}
+    else:
+        res = {"workload": wl.name, "mla_attention": run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl,
+                                                                     flush, pk)}
     if rank == 0:
-        print(json.dumps({"workload": wl.name, "mla_attention": res}), flush=True)
+        print(json.dumps(res), flush=True)
 
 
 def run_ours(args, wl, world, rank, local):
@@ -466,6 +523,7 @@ def run_ours(args, wl, world, rank, local):
     e2e_ms = run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world)
     proj = None if args.no_projections else run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush,
                                                               peaks()[0])
+    sparse = None if args.no_sparse else run_sparse(args, dev, flush, peaks()[0])
     h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
 
@@ -509,6 +567,8 @@ def run_ours(args, wl, world, rank, local):
             "gpu_launches": 3 * K}
     if proj is not None:
         line["mla_attention"] = proj
+    if sparse is not None:
+        line["sparse_decode"] = sparse
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10 s of oracle work: the sample repeated until 10 s have passed
         n_req = max(1, min(wl.batch, args.ref_requests))
@@ -535,6 +595,8 @@ def main():
                     help="skip the timing of the query absorption / output decompression kernels")
     ap.add_argument("--projections-only", action="store_true",
                     help="time only the query absorption / output decompression kernels and the whole step")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the timing of the token-level sparse decode")
+    ap.add_argument("--sparse-only", action="store_true", help="time only the token-level sparse decode")
     ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
     ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,
@@ -545,7 +607,7 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, wl, world, rank)
-        elif args.projections_only:
+        elif args.projections_only or args.sparse_only:
             run_projections_only(args, wl, world, rank)
         else:
             run_ours(args, wl, world, rank, local)
