@@ -355,15 +355,29 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
                                   "frac": gbs / pk["hbm_gbs"],
                                   "frac_net_of_empty_launch": by / (net * 1e-6) / 1e9 / pk["hbm_gbs"]}}
     chain_us = timed(chain)
+    # the same chain captured once in a CUDA graph and replayed (launch work
+    # on the host leaves the timed region; the device work is unchanged)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        chain()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        chain()
+    graph_us = timed(graph.replay)
+    del graph
     if int(status.item()) != 0 or dec.status() != 0:
         raise RuntimeError("device status set in the projection timing")
     flops, _ = cost.workload_cost(wl)
     res["whole_step_us"] = chain_us
+    res["whole_step_graph_us"] = graph_us
     res["whole_step"] = "absorb -> schedule -> decode -> combine -> decompress, one event pair around it"
     res["whole_step_tflops"] = (flops + 2 * 2 * R * h * 128 * 512) / (chain_us * 1e-6) / 1e12
     res["rows"], res["heads"] = R, h
-    # timed launches: absorb alone, decompress alone, and the chain's five kernels
-    res["gpu_launches"] = args.steps * (1 + 1 + 5)
+    # timed launches: absorb alone, decompress alone, and the chain's five kernels (twice: launched, replayed)
+    res["gpu_launches"] = args.steps * (1 + 1 + 5 + 5)
     return res
 
 
