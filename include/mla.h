@@ -201,24 +201,25 @@ int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, const void* 
  * A position outside [0, seqlens[r]) (e.g. -1 padding) is skipped; a
  * position listed twice is two keys; a list with no valid position gives
  * O = 0 and lse = -inf.  Positions resolve through block_table as for the
- * dense decode.  Supported: BF16 cache, causal = 0 (the lists decide what
- * each query token sees).  The selected rows are gathered into scratch pages
- * of the workspace, then the tensor-core decode runs over them.
- *   shape, q, kv_cache, block_table, seqlens, out, lse: as for mla_decode_fwd.
+ * dense decode.  Both cache types; causal must be 0 (the lists decide what
+ * each query token sees).  The selected rows (FP8: with their scales) are
+ * gathered into scratch pages of the workspace, in the cache's own page
+ * format, then the tensor-core decode runs over them.
+ *   shape, q, kv_cache, kv_scale, block_table, seqlens, out, lse: as for
+ *             mla_decode_fwd (kv_scale NULL for a BF16 cache).
  *   topk    : list length per query token, 1 <= topk <= 2^24.
  *   indices : device int32 [batch, s_q, topk], 4-byte aligned.
  *   workspace: device buffer of mla_sparse_workspace_bytes(shape, topk,
  *             num_sms of this device) bytes, 256-byte aligned, zero-filled
  *             before its first use (it holds the status word); the caller
  *             must not touch it while the call's work runs.
- * Returns MLA_ERR_UNSUPPORTED for an FP8 cache or a shape whose b*s_q*
- * ceil(topk/64) scratch pages exceed 2^31; MLA_ERR_WORKSPACE when
- * workspace_bytes is too small. */
+ * Returns MLA_ERR_UNSUPPORTED for a shape whose b*s_q*ceil(topk/64) scratch
+ * pages reach 2^26; MLA_ERR_WORKSPACE when workspace_bytes is too small. */
 size_t mla_sparse_workspace_bytes(const mla_shape_t* shape, int topk, int num_sms);
 int mla_sparse_decode_fwd(const mla_shape_t* shape, int topk, const void* q, const void* kv_cache,
-                          const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
-                          float softmax_scale, void* workspace, size_t workspace_bytes, void* out, float* lse,
-                          void* stream);
+                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens,
+                          const int32_t* indices, float softmax_scale, void* workspace, size_t workspace_bytes,
+                          void* out, float* lse, void* stream);
 /* Device status of the sparse decode's kernels (bounded waits, out-of-range
  * lengths or page ids); as mla_get_device_status, SYNCHRONISES `stream`. */
 int mla_sparse_get_device_status(const mla_shape_t* shape, int topk, int num_sms, void* workspace, void* stream,

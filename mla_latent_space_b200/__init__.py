@@ -74,7 +74,7 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_noalloc.restype = i32
         L.mla_sparse_workspace_bytes.argtypes = [sp, i32, i32]
         L.mla_sparse_workspace_bytes.restype = sz
-        L.mla_sparse_decode_fwd.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp, sz, vp, vp, vp]
+        L.mla_sparse_decode_fwd.argtypes = [sp, i32, vp, vp, vp, vp, vp, vp, f32, vp, sz, vp, vp, vp]
         L.mla_sparse_decode_fwd.restype = i32
         L.mla_sparse_get_device_status.argtypes = [sp, i32, i32, vp, vp, ctypes.POINTER(i32)]
         L.mla_sparse_get_device_status.restype = i32
@@ -250,14 +250,16 @@ class SparseDecoder:
         self.n_sms = num_sms(self.device)
         nb = mla_sparse_workspace_bytes(shape, self.topk, self.n_sms)
         if nb == 0:
-            raise MLAError(-2, "SparseDecoder: shape not supported (BF16 cache, causal=0, topk >= 1)")
+            raise MLAError(-2, "SparseDecoder: shape not supported (causal=0, topk >= 1)")
         self.workspace = torch.zeros(nb, dtype=torch.uint8, device=self.device)
 
-    def decode(self, q, kv_cache, block_table, seqlens, indices, softmax_scale, out, lse, stream=None):
+    def decode(self, q, kv_cache, block_table, seqlens, indices, softmax_scale, out, lse, stream=None,
+               kv_scale=None):
         sh = self.shape
-        _check_decode_tensors(sh, q, kv_cache, None, block_table, seqlens, out, lse)
+        _check_decode_tensors(sh, q, kv_cache, kv_scale, block_table, seqlens, out, lse)
         _need(indices, "indices", torch.int32, (sh.batch, sh.s_q, self.topk))
-        rc = lib().mla_sparse_decode_fwd(ctypes.byref(sh), self.topk, _ptr(q), _ptr(kv_cache), _ptr(block_table),
+        rc = lib().mla_sparse_decode_fwd(ctypes.byref(sh), self.topk, _ptr(q), _ptr(kv_cache), _ptr(kv_scale),
+                                         _ptr(block_table),
                                          _ptr(seqlens), _ptr(indices), float(softmax_scale), _ptr(self.workspace),
                                          self.workspace.numel(), _ptr(out), _ptr(lse), _stream(stream))
         _check(rc, "mla_sparse_decode_fwd")

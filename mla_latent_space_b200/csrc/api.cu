@@ -23,8 +23,8 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
                         void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
 cudaError_t launch_sparse_gather(const int32_t* indices, int topk, const int32_t* seqlens, int batch, int s_q,
                                  const int32_t* block_table, int max_pages, int num_pages, const void* pool,
-                                 void* scratch, int vpages, int32_t* vseqlens, int32_t* vbt, void* status_ws,
-                                 cudaStream_t stream);
+                                 const float* kv_scale, void* scratch, float* vscale, int vpages, int32_t* vseqlens,
+                                 int32_t* vbt, void* status_ws, bool fp8, cudaStream_t stream);
 int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* qz, int32_t* status,
                     cudaStream_t stream);
 int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
@@ -109,20 +109,22 @@ int check_decode_args(const mla_shape_t* shape, const void* q, const void* kv, c
 
 // Workspace of the sparse decode (every region 256-byte aligned): the
 // compacted lengths and identity block table of the b*s single-query
-// "virtual" requests, their schedule, the decode workspace, and the scratch
-// pages the selected rows are gathered into.
+// "virtual" requests, their schedule, the decode workspace, the scratch
+// pages the selected rows are gathered into (the cache's own page format)
+// and, for the FP8 cache, their per-token scales.
 struct SparseLayout {
   mla_shape_t vshape;
   int vpages;
-  size_t vseq, vbt, sched, sched_bytes, ws, ws_bytes, scratch, total;
+  size_t vseq, vbt, sched, sched_bytes, ws, ws_bytes, scratch, vscale, total;
 };
 
 bool sparse_layout(const mla_shape_t* s, int topk, int num_sms, SparseLayout* L) {
   if (check_shape(s) != MLA_OK || topk < 1 || topk > (1 << 24) || num_sms < 1) return false;
-  if (s->cache_dtype != MLA_CACHE_BF16 || s->causal != 0) return false;
+  if (s->causal != 0) return false;
+  const bool fp8 = s->cache_dtype == MLA_CACHE_FP8_E4M3;
   const int64_t V = int64_t(s->batch) * s->s_q;
   const int64_t vpages = (topk + MLA_PAGE_SIZE - 1) / MLA_PAGE_SIZE;
-  if (V * vpages >= (int64_t(1) << 31)) return false;
+  if (V * vpages >= (int64_t(1) << 26)) return false;   // scratch rows stay below 2^32
   mla_shape_t vs = *s;
   vs.batch = int32_t(V);
   vs.s_q = 1;
@@ -145,7 +147,11 @@ bool sparse_layout(const mla_shape_t* s, int topk, int num_sms, SparseLayout* L)
   L->ws_bytes = kStatusBytes + size_t(max_slots_for(num_workers_for(num_sms))) * kSlotBytes;
   off = up(off + L->ws_bytes);
   L->scratch = off;
-  off += size_t(V) * size_t(vpages) * MLA_PAGE_SIZE * (2 * MLA_D_QK);
+  const size_t page_bytes = fp8 ? size_t(MLA_PAGE_SIZE) * (MLA_D_V + 2 * MLA_D_ROPE)
+                                : size_t(MLA_PAGE_SIZE) * (2 * MLA_D_QK);
+  off = up(off + size_t(V) * size_t(vpages) * page_bytes);
+  L->vscale = off;
+  if (fp8) off = up(off + size_t(V) * size_t(vpages) * MLA_PAGE_SIZE * 4);
   L->total = off;
   return true;
 }
@@ -251,15 +257,16 @@ size_t mla_sparse_workspace_bytes(const mla_shape_t* shape, int topk, int num_sm
 }
 
 int mla_sparse_decode_fwd(const mla_shape_t* shape, int topk, const void* q, const void* kv_cache,
-                          const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
-                          float softmax_scale, void* workspace, size_t workspace_bytes, void* out, float* lse,
-                          void* stream) {
+                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens,
+                          const int32_t* indices, float softmax_scale, void* workspace, size_t workspace_bytes,
+                          void* out, float* lse, void* stream) {
   int rc = check_shape(shape);
   if (rc != MLA_OK) return rc;
-  if (shape->cache_dtype != MLA_CACHE_BF16) return MLA_ERR_UNSUPPORTED;
+  const bool fp8 = shape->cache_dtype == MLA_CACHE_FP8_E4M3;
   if (shape->causal != 0 || topk < 1 || topk > (1 << 24)) return MLA_ERR_INVALID_ARG;
   if (!q || !kv_cache || !block_table || !seqlens || !indices || !workspace || !out || !lse)
     return MLA_ERR_INVALID_ARG;
+  if (fp8 && (!kv_scale || !aligned(kv_scale, 4))) return MLA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(kv_cache, 256) || !aligned(out, 16) || !aligned(lse, 4) ||
       !aligned(block_table, 4) || !aligned(seqlens, 4) || !aligned(indices, 4) || !aligned(workspace, 256))
     return MLA_ERR_INVALID_ARG;
@@ -275,15 +282,17 @@ int mla_sparse_decode_fwd(const mla_shape_t* shape, int topk, const void* q, con
   void* sched = w + L.sched;
   void* ws = w + L.ws;
   void* scratch = w + L.scratch;
+  float* vscale = fp8 ? reinterpret_cast<float*>(w + L.vscale) : nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (launch_sparse_gather(indices, topk, seqlens, shape->batch, shape->s_q, block_table, shape->max_pages_per_seq,
-                           shape->num_pages, kv_cache, scratch, L.vpages, vseq, vbt, ws, st) != cudaSuccess)
+                           shape->num_pages, kv_cache, kv_scale, scratch, vscale, L.vpages, vseq, vbt, ws, fp8,
+                           st) != cudaSuccess)
     return MLA_ERR_CUDA;
   const ShapeInfo si = shape_info(&L.vshape);
   if (launch_schedule(vseq, si, num_workers_for(sms), static_cast<int32_t*>(sched), st) != cudaSuccess)
     return MLA_ERR_CUDA;
   const int cap = cap_slots_for(L.ws_bytes);
-  rc = launch_decode_sm100(&L.vshape, q, scratch, nullptr, vbt, vseq, softmax_scale, sched, ws, cap, out, lse, st);
+  rc = launch_decode_sm100(&L.vshape, q, scratch, vscale, vbt, vseq, softmax_scale, sched, ws, cap, out, lse, st);
   if (rc != MLA_OK) return rc;
   return launch_combine(sched, ws, out, lse, si.batch * si.tiles_per_req, cap, st) == cudaSuccess ? MLA_OK
                                                                                                   : MLA_ERR_CUDA;

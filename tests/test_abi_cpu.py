@@ -109,17 +109,21 @@ def test_sparse_workspace_and_argument_checks():
     # virtual requests: 64 x 32 scratch pages of 73,728 B, plus lengths, block table, schedule, decode workspace
     nb = mla.mla_sparse_workspace_bytes(s, 2048, 148)
     assert 64 * 32 * 73728 < nb < 64 * 32 * 73728 + (64 << 20)
-    assert mla.mla_sparse_workspace_bytes(mla.make_shape(64, 1, 128, 512, 32768, cache_dtype="fp8"), 2048, 148) == 0
+    # FP8: 40,960-byte scratch pages plus 64 fp32 scales per page
+    nb8 = mla.mla_sparse_workspace_bytes(mla.make_shape(64, 1, 128, 512, 32768, cache_dtype="fp8"), 2048, 148)
+    assert 64 * 32 * (40960 + 256) < nb8 < 64 * 32 * (40960 + 256) + (64 << 20)
     assert mla.mla_sparse_workspace_bytes(mla.make_shape(4, 2, 128, 8, 64, causal=True), 64, 148) == 0
     assert mla.mla_sparse_workspace_bytes(s, 0, 148) == 0
     L = mla.lib()
     fake = ctypes.c_void_p(1 << 20)
-    args = lambda sh, k, idx=fake, q=fake: (ctypes.byref(sh), k, q, fake, fake, fake, idx, 0.1, fake, 1 << 40, fake,
-                                            fake, None)
+    args = lambda sh, k, idx=fake, q=fake, sc=None: (ctypes.byref(sh), k, q, fake, sc, fake, fake, idx, 0.1, fake,
+                                                     1 << 40, fake, fake, None)
     assert L.mla_sparse_decode_fwd(*args(s, 2048, idx=None)) == -1
     assert L.mla_sparse_decode_fwd(*args(s, 2048, q=ctypes.c_void_p((1 << 20) + 8))) == -1
     assert L.mla_sparse_decode_fwd(*args(s, 0)) == -1
-    assert L.mla_sparse_decode_fwd(*args(mla.make_shape(64, 1, 128, 512, 32768, cache_dtype="fp8"), 2048)) == -2
+    assert L.mla_sparse_decode_fwd(*args(mla.make_shape(64, 1, 128, 512, 32768, cache_dtype="fp8"), 2048)) == -1
+    assert L.mla_sparse_decode_fwd(*args(mla.make_shape(64, 1, 128, 512, 32768, cache_dtype="fp8"), 2048,
+                                         sc=ctypes.c_void_p((1 << 20) + 2))) == -1
     assert L.mla_sparse_decode_fwd(*args(mla.make_shape(4, 2, 128, 8, 64, causal=True), 64)) == -1
 
 

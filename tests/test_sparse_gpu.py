@@ -23,7 +23,7 @@ def _built():
 
 
 def run_sparse(wl, idx, poison_out=True):
-    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages)
+    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages, wl.cache_dtype)
     dec = mla.SparseDecoder(shape, idx.shape[-1])
     out = torch.empty((wl.batch, wl.s_q, wl.num_heads, 512), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((wl.batch, wl.s_q, wl.num_heads), dtype=torch.float32, device="cuda")
@@ -31,7 +31,8 @@ def run_sparse(wl, idx, poison_out=True):
         out.fill_(float("nan"))
         lse.fill_(float("nan"))
     dec.decode(wl.q.cuda(), wl.pool.cuda(), torch.from_numpy(wl.block_table).cuda(),
-               torch.from_numpy(wl.seqlens).cuda(), torch.from_numpy(idx).cuda(), wl.softmax_scale, out, lse)
+               torch.from_numpy(wl.seqlens).cuda(), torch.from_numpy(idx).cuda(), wl.softmax_scale, out, lse,
+               kv_scale=None if wl.kv_scale is None else wl.kv_scale.cuda())
     torch.cuda.synchronize()
     return out.float().cpu().numpy(), lse.cpu().numpy(), dec.status()
 
@@ -103,3 +104,18 @@ def test_sparse_bench_shape_sampled():
                       kv_scale=None, softmax_scale=wl.softmax_scale)
     O_ref, L_ref = oracle.sparse_decode(sub, idx[rs])
     assert_parity(compare(O[rs], L[rs], O_ref, L_ref), "sparse_bench_sampled")
+
+
+def test_sparse_fp8_random_lists_with_padding_and_out_of_range():
+    wl = mw.make(3, 2, 128, [300, 70, 1000], cache_dtype="fp8", seed=61, name="sparse_fp8")
+    idx = mw.make_sparse_indices(wl.seqlens, 2, 100, seed=62, pad=10)
+    idx[0, 1, 90] = idx[0, 1, 0]            # a repeated position
+    idx[1, 0, 91] = 70                      # one past the end: skipped
+    idx[2, 1, 92] = 999                     # the last token
+    check(wl, idx)
+
+
+@pytest.mark.parametrize("topk", [1, 65, 700])
+def test_sparse_fp8_list_lengths(topk):
+    wl = mw.make(2, 1, 128, [500, 4000], cache_dtype="fp8", seed=63, name=f"sparse_fp8_k{topk}")
+    check(wl, mw.make_sparse_indices(wl.seqlens, 1, topk, seed=64))
