@@ -376,6 +376,18 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
     res["whole_step"] = "absorb -> schedule -> decode -> combine -> decompress, one event pair around it"
     res["whole_step_tflops"] = (flops + 2 * 2 * R * h * 128 * 512) / (chain_us * 1e-6) / 1e12
     res["rows"], res["heads"] = R, h
+    if not args.no_cpu_baseline:
+        # the fp64 oracle's two projections on the same inputs, on the host cores
+        import oracle
+        f64 = oracle.bf16_to_f64
+        qf, wkf, of, wvf = f64(p.q), f64(p.w_k), f64(p.o_lat), f64(p.w_kvb2)
+        t0 = time.perf_counter()
+        oracle.absorb(qf, wkf)
+        t1 = time.perf_counter()
+        oracle.decompress(of, wvf)
+        t2 = time.perf_counter()
+        res["cpu_baseline"] = {"kind": "oracle", "cores": blas_threads(), "absorb_us": (t1 - t0) * 1e6,
+                               "decompress_us": (t2 - t1) * 1e6, "sample": f"all {R} rows x {h} heads"}
     # timed launches: absorb alone, decompress alone, and the chain's five kernels (twice: launched, replayed)
     res["gpu_launches"] = args.steps * (1 + 1 + 5 + 5)
     return res
@@ -425,13 +437,27 @@ def run_sparse(args, dev, flush, pk):
     flops, nbytes = sparse_cost(wl.batch, wl.s_q, wl.num_heads, S["topk"])
     gbs = nbytes / (us * 1e-6) / 1e9
     del pool
+    cpu = None
+    if not args.no_cpu_baseline:
+        # the fp64 oracle on the first two requests, scaled to a whole call
+        import oracle
+        n = 2
+        sub = mw.Workload(name="sub", batch=n, s_q=wl.s_q, num_heads=wl.num_heads, causal=False, cache_dtype="bf16",
+                          seqlens=wl.seqlens[:n], block_table=wl.block_table[:n], q=wl.q[:n], pool=wl.pool,
+                          kv_scale=None, softmax_scale=wl.softmax_scale)
+        t0 = time.perf_counter()
+        oracle.sparse_decode(sub, idx[:n])
+        dt = time.perf_counter() - t0
+        cpu = {"kind": "oracle", "cores": blas_threads(), "us_per_call": dt * 1e6 * wl.batch / n,
+               "tflops": flops * n / wl.batch / dt / 1e12,
+               "sample": f"{n} of {wl.batch} requests (each gathers its whole cache in fp64), scaled to the call"}
     return {"workload": wl.name, "topk": S["topk"], "us_per_call": us, "tflops": flops / (us * 1e-6) / 1e12,
             "kernels": "gather -> schedule -> decode -> combine (4 launches)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "bytes": nbytes,
                          "note": "bytes of a fused design (each listed row read once); this composition moves "
                                  "each row three times"},
-            "gpu_launches": 4 * args.steps}
+            "gpu_launches": 4 * args.steps, "cpu_baseline": cpu}
 
 
 def run_projections_only(args, wl, world, rank):
