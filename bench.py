@@ -42,14 +42,14 @@ L2_FLUSH_BYTES = 256 << 20
 # were taken on: reported as null as soon as any of them differs (checked by
 # content hash at run time).
 TRAFFIC_SOURCES_SHA1 = {
-    "mla_latent_space_b200/csrc/decode_sm100.cu": "9f355e13e78226a1ceb429fc78162d6330de39ab",
+    "mla_latent_space_b200/csrc/decode_sm100.cu": "63cd7bb64378a3a73db3b85da200e0e53e9f224d",
     "mla_latent_space_b200/csrc/sm100_ptx.cuh": "a666c6fb95adecc45850f281b1be3ecacba5d16c",
     "mla_latent_space_b200/csrc/kernel_util.cuh": "c304dedb0965e65632e557168f97693bf2077cdb",
-    "mla_latent_space_b200/csrc/common.cuh": "0bfcb7c010a0345f9ee30813ac952b25f0c1d15d",
+    "mla_latent_space_b200/csrc/common.cuh": "1bda35f3e244dc99d70c2901283243f600e444f6",
 }
 TRAFFIC_BYTES = {   # profiles/decode_sm100_dsv3_b64_h128_t4096.md, profiles/decode_sm100_fp8_b64_h128_t32768.md
-    "dsv3_b64_h128_t4096_paged": 311.552256e6 + 5.468160e6,
-    "fp8_b64_h128_t32768": 1369.464e6 + 21.736448e6,
+    "dsv3_b64_h128_t4096_paged": 311.547136e6 + 4.920576e6,
+    "fp8_b64_h128_t32768": 1374.59968e6 + 23.452416e6,
 }
 
 

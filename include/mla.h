@@ -127,10 +127,10 @@ int mla_get_schedule(const mla_shape_t* shape, const int32_t* seqlens, int num_s
  *                The tensor-core kernel (tcgen05, 2-SM clusters) rounds P to
  *                fp16 and converts V to fp16 on chip, so value rows must lie
  *                within fp16 range (|v| < 65504; FP8: |e4m3 * scale|).  FP8
- *                cache: the latent scores use e4m3 -> fp16 (exact) against an
- *                fp16 copy of the query's latent part, so those query values
- *                must lie within fp16 range too; a value outside it is flagged
- *                (MLA_ERR_DEVICE_CHECK from mla_get_device_status).
+ *                cache: the latent scores multiply the cache's e4m3 values
+ *                directly with a two-part e4m3 copy of the query's latent
+ *                part (per-row power-of-two scale), which holds every bf16
+ *                query value exactly down to 2^-11 of its row's largest.
  *   lse        : fp32 [batch, s_q, num_heads], natural-log log-sum-exp of the
  *                scaled scores (-inf for a row that sees no key).
  * Tiles cut into several pieces are finished by mla_combine; tiles in one

@@ -58,11 +58,10 @@ using namespace ptx;
 // of both pages (the ninth box, the RoPE columns, alone in the fifth), so
 // the QK issuer waits once per 8 MMAs: each wait in the issuing thread idles
 // the tensor pipe, whose queue holds only a few MMAs.  FP8 cache: 6 stages
-// of 16 KB (e4m3 and RoPE stages).
+// of 16 KB (query, e4m3 and RoPE stages; 10 measured no faster).
 constexpr int NZ = 5;
 constexpr int NZ8 = 6;
 constexpr int kNZMax = 6;
-constexpr int NC = 4;   // FP8 cache: 16 KB stages of fp16 cache rows converted from e4m3
 // P page slots (output CTA): slot 0 takes page 0 of a block with the block's
 // rescale factors and row sums, slot 1 its page 1.  Each is refilled as soon
 // as its own page's PVs completed, so the next block's page 0 crosses over
@@ -95,14 +94,14 @@ constexpr int kConvThreads = 256;                     // output-CTA converter wa
 constexpr int kSmThreads = 256;                       // score-CTA warps 4..11
 constexpr uint32_t kSoftmaxBar = 1;                   // named barrier of the softmax warps
 constexpr uint32_t kConvBar = 2;                      // named barrier of a CTA's converter warps
-constexpr int kConvThreadsS = 192;                    // FP8 cache: score-CTA converters, warps 2, 3, 12..15
 constexpr uint32_t kFp8PageBytes = 64 * 512 + 64 * 64 * 2;   // 64x512 e4m3, then 64x64 bf16 RoPE
 constexpr uint32_t kTmemSLat = 256;                   // FP8 cache: latent-part scores, columns 256..383
+constexpr uint32_t kTmemQLo = 128;                    // FP8 cache: the query's e4m3 lo part, columns 128..255
 
 struct Bars {
-  // score CTA (FP8 cache: also the converted ring and the query RoPE buffer)
+  // score CTA (FP8 cache: also the query RoPE buffer)
   uint64_t z_full[kNZMax], z_empty[kNZMax], s_full, s_empty, q_ready, x_free[NX];
-  uint64_t c_full[NC], c_empty[NC], qpe_full, qpe_empty;
+  uint64_t qpe_full, qpe_empty;
   // output CTA
   uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_go, corr_done, pv_blk[NB], o_free;
   // correction events, from the PV issuer warp to the correction warpgroup:
@@ -118,19 +117,20 @@ struct Bars {
 
 constexpr uint32_t kOffData = 1024;
 // score CTA.  BF16 cache: ring | P staging | exchange.  FP8 cache: ring |
-// converted ring | query RoPE columns (128 rows x 64, one 16 KB stage) |
-// P staging | exchange | per-token scales of the block's two pages.
+// query RoPE columns (128 rows x 64, one 16 KB stage) | P staging |
+// exchange | per-token scales of the block's two pages | half-row maxima of
+// the query.
 template <bool kFp8>
 struct LayS {
   static constexpr int nz = kFp8 ? NZ8 : NZ;
   static constexpr uint32_t zbytes = kFp8 ? kZStage : 2 * kZStage;   // bytes per ring stage
   static constexpr uint32_t z = kOffData;
-  static constexpr uint32_t c = z + nz * zbytes;
-  static constexpr uint32_t qpe = c + (kFp8 ? NC * kZStage : 0u);
+  static constexpr uint32_t qpe = z + nz * zbytes;
   static constexpr uint32_t stage = qpe + (kFp8 ? kZStage : 0u);
   static constexpr uint32_t xchg = stage + kPStage;               // row max / sum exchange
   static constexpr uint32_t scales = xchg + 4 * 128 * 4;           // FP8: 2 x 64 fp32
-  static constexpr uint32_t end = scales + (kFp8 ? 2 * 64 * 4 : 0u);
+  static constexpr uint32_t qam = scales + (kFp8 ? 2 * 64 * 4 : 0u);   // FP8: 2 x 128 fp32 half-row maxima
+  static constexpr uint32_t end = qam + (kFp8 ? 2 * 128 * 4 : 0u);
 };
 constexpr uint32_t kSmemS = LayS<false>::end > LayS<true>::end ? LayS<false>::end : LayS<true>::end;
 // output CTA
@@ -142,7 +142,7 @@ static_assert(sizeof(Bars) <= kOffData, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kPSlot0 % 1024 == 0 && kPStage % 1024 == 0 && kZStage % 1024 == 0,
               "swizzle atoms need 1024-byte alignment");
-static_assert(LayS<true>::c % 1024 == 0 && LayS<true>::qpe % 1024 == 0 && LayS<true>::stage % 1024 == 0, "align");
+static_assert(LayS<true>::qpe % 1024 == 0 && LayS<true>::stage % 1024 == 0, "align");
 
 // Instruction descriptors (kind::f16, fp32 accumulate, M = 128).
 //   QK: A = Q bf16 (TMEM), B = cache rows bf16 K-major, N = 128
@@ -150,8 +150,9 @@ static_assert(LayS<true>::c % 1024 == 0 && LayS<true>::qpe % 1024 == 0 && LayS<t
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((256u >> 3) << 17) |
                               ((128u >> 4) << 24);
-//   FP8 cache, latent part: A = Q fp16 (TMEM), B = converted rows fp16 K-major, N = 128
-constexpr uint32_t kIdescQKh = (1u << 4) | (0u << 7) | (0u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+//   FP8 cache, latent part (kind::f8f6f4): A = the query's e4m3 hi or lo part
+//   (TMEM), B = the cache's e4m3 rows K-major, N = 128
+constexpr uint32_t kIdescQK8 = (1u << 4) | (0u << 7) | (0u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 // Shared-memory matrix descriptor, 128-byte swizzle.  lbo / sbo in bytes.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -329,11 +330,54 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two, __half2 scale) {
 
 // bf16 pair -> fp16 pair (exact inside fp16's range); *big records a value
 // outside it (or NaN).
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2_checked(uint32_t w, bool* big) {
-  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-  *big |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f8f6f4 (the FP8 cache's latent scores).
+__device__ __forceinline__ void mma_ts_f8(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's lane (32x32b shape).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Largest |value| of the two bf16 values of w.
+__device__ __forceinline__ float bf16_abs_max(uint32_t w) {
+  return fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xFFFF0000u)));
+}
+
+// e with am / 2^e <= 448 (e4m3's largest finite value), smallest such; 0
+// for am = 0 or a non-finite am (its NaN or infinity then reaches S as is).
+__device__ __forceinline__ int pow2_scale_exp(float am) {
+  if (!(am > 0.f) || !(am <= 3.402823466e38f)) return 0;
+  int e = int(ceilf(log2f(am * (1.f / 448.f))));
+  while (ldexpf(am, -e) > 448.f) ++e;        // log2f's rounding, either way
+  while (ldexpf(am, -(e - 1)) <= 448.f) --e;
+  return e;
+}
+
+// Four bf16 values (w01, w23, low half first) times `inv` (a power of two)
+// as e4m3 hi = RNE(x) and lo = RNE(x - hi), four bytes each, value 4k+j in
+// byte j.  x - hi is exact in fp32.
+__device__ __forceinline__ void split_e4m3x4(uint32_t w01, uint32_t w23, float inv, uint32_t* hi, uint32_t* lo) {
+  const float2 a = make_float2(__uint_as_float(w01 << 16) * inv, __uint_as_float(w01 & 0xFFFF0000u) * inv);
+  const float2 b = make_float2(__uint_as_float(w23 << 16) * inv, __uint_as_float(w23 & 0xFFFF0000u) * inv);
+  const __nv_fp8x2_storage_t ha = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hb = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
+  const float2 fa = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(ha, __NV_E4M3)));
+  const float2 fb = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hb, __NV_E4M3)));
+  const __nv_fp8x2_storage_t la = __nv_cvt_float2_to_fp8x2(make_float2(a.x - fa.x, a.y - fa.y), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t lb = __nv_cvt_float2_to_fp8x2(make_float2(b.x - fb.x, b.y - fb.y), __NV_SATFINITE, __NV_E4M3);
+  *hi = uint32_t(ha) | (uint32_t(hb) << 16);
+  *lo = uint32_t(la) | (uint32_t(lb) << 16);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -405,11 +449,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   [[maybe_unused]] unsigned trk_ = 0;   // trace builds: this thread's event count (one recording thread per role)
 
   if (tid == 0) {
-    // FP8 cache: a ring stage is refilled once the softmax, the issuer and
-    // the converters have each released it (see the issuer)
+    // FP8 cache: a ring stage is refilled once the softmax and the issuer
+    // have each released it (see the issuer)
     for (int s = 0; s < kNZMax; ++s) {
       mbar_init(bar(bars->z_full[s]), 1);
-      mbar_init(bar(bars->z_empty[s]), kFp8 ? 3 : 1);
+      mbar_init(bar(bars->z_empty[s]), kFp8 ? 2 : 1);
     }
     mbar_init(bar(bars->s_full), 1);
     mbar_init(bar(bars->s_empty), kSmThreads);
@@ -426,10 +470,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       mbar_init(bar(bars->pv_done[s]), 1);
     }
     for (int s = 0; s < NB; ++s) mbar_init(bar(bars->pv_blk[s]), 1);
-    for (int s = 0; s < NC; ++s) {
-      mbar_init(bar(bars->c_full[s]), kConvThreadsS);
-      mbar_init(bar(bars->c_empty[s]), 1);
-    }
     mbar_init(bar(bars->qpe_full), 1);
     mbar_init(bar(bars->qpe_empty), 1);
     mbar_init(bar(bars->o_free), 128);
@@ -598,22 +638,21 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     } else if (warp == 1) {
       // ---- QK^T issuer warp: per block 36 MMAs M128 N128 K16.  BF16 cache: 5
       // stages of 2 boxes (the last 1) x 4 MMAs, A = Q (TMEM), into S.  FP8 cache: the RoPE stage x 4 with
-      // A = the query RoPE columns (shared memory) into S_rope, then 8
-      // converted fp16 stages x 4 with A = the fp16 query (TMEM) into S_lat.
+      // A = the query RoPE columns (shared memory) into S_rope, then the 4
+      // e4m3 stages x (4 + 4) kind::f8f6f4 MMAs with A = the query's e4m3 hi
+      // and lo parts (TMEM) into S_lat.
       // The warp waits and computes operands together; one lane issues.
       const bool leader = elect_one();
       const uint64_t zdesc0 = sdesc(sbase + L::z, 16, 1024);
-      const uint64_t cdesc0 = sdesc(sbase + L::c, 16, 1024);
       const uint64_t qdesc = sdesc(sbase + L::qpe, 16, 1024);
-      uint32_t zc = 0, cc = 0, bc = 0, pieces = 0;
+      uint32_t zc = 0, bc = 0, pieces = 0;
       each_piece(sv, [&](const Piece& pc) {
         // FP8 cache: the ring is shorter than the query, so its stages are
-        // released one by one.  This warp and one converter thread walk
-        // every stage of the ring in order (a parity wait is only sound when
-        // the stage's previous use has completed), and a stage is refilled
-        // after three releases: softmax, issuer, converter.  For the RoPE
-        // and e4m3 stages, which the softmax never sees, the issuer releases
-        // twice.
+        // released one by one.  This warp walks every stage of the ring in
+        // order (a parity wait is only sound when the stage's previous use
+        // has completed), and a stage is refilled after two releases: softmax
+        // and issuer.  For the RoPE and e4m3 stages, which the softmax never
+        // sees, the issuer releases twice.
         constexpr int nq = kFp8 ? 8 : 5;   // ring stages of the query
         if constexpr (kFp8) {
           for (int u = 0; u < nq; ++u, ++zc) {
@@ -655,24 +694,23 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               __syncwarp();
               ++zc;
             }
-            for (int c = 0; c < 8; ++c, ++cc) {
-              if ((c & 1) == 0) {   // e4m3 stage c/2: observed in order, released for issuer and softmax
-                if (!ewait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u)) return false;
-                if (leader) mbar_arrive_cnt(bar(bars->z_empty[zc % nz]), 2u);
-                ++zc;
-              }
-              const uint32_t cs = cc % NC;
-              if (!ewait(ctl, bar(bars->c_full[cs]), (cc / NC) & 1u)) return false;
-              if (leader) MLA_TR(1, 21, cc);
+            // the four e4m3 stages, straight from the cache: S_lat =
+            // Q_hi . K + Q_lo . K, 4 + 4 MMAs of K = 32 per stage
+            for (int e = 0; e < 4; ++e, ++zc) {
+              const uint32_t zs = zc % nz;
+              if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
+              if (leader) MLA_TR(1, 21, zc);
               tc_fence_after();
-              const uint64_t bd = cdesc0 + uint64_t(cs * (kZStage >> 4));
-              const uint32_t ad = tmem + 32u * c, d = tmem + kTmemSLat;
+              const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
+              const uint32_t d = tmem + kTmemSLat;
               if (leader) {
-                mma_ts(d, ad, bd, kIdescQKh, c != 0);
-                mma_ts(d, ad + 8u, bd + 2u, kIdescQKh, 1u);
-                mma_ts(d, ad + 16u, bd + 4u, kIdescQKh, 1u);
-                mma_ts(d, ad + 24u, bd + 6u, kIdescQKh, 1u);
-                mma_commit(bar(bars->c_empty[cs]));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  mma_ts_f8(d, tmem + 32u * e + 8u * k, bd + 2u * k, kIdescQK8, (e | k) != 0 ? 1u : 0u);
+                  mma_ts_f8(d, tmem + kTmemQLo + 32u * e + 8u * k, bd + 2u * k, kIdescQK8, 1u);
+                }
+                mma_commit(bar(bars->z_empty[zs]));    // the issuer's release, when the MMAs are done
+                mbar_arrive(bar(bars->z_empty[zs]));   // the softmax's
               }
               __syncwarp();
             }
@@ -714,75 +752,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       if (leader) mma_commit(bar(bars->mma_done));
       __syncwarp();
       drain_wait(bar(bars->mma_done), 0);
-    } else if (kFp8 && (warp == 2 || warp == 3 || warp >= 12)) {
-      // ---- FP8 cache: converters.  Each e4m3 stage (128 latent columns of
-      // the block's two pages) becomes two fp16 stages of 64 columns in the
-      // K-major 128-byte-swizzled layout of the bf16 path.  e4m3 -> fp16 is
-      // exact.  Six warps (2, 3 and 12-15): four left the stages' latency
-      // exposed.
-      const int t = (warp < 12 ? warp - 2 : warp - 10) * 32 + lane;
-      // chunk o (16 e4m3 values) is row o / 8 of the stage (page row / 64,
-      // token row % 64), 16-byte column o % 8; thread t takes o = t + 192u
-      constexpr int kCh = (128 * 8 + kConvThreadsS - 1) / kConvThreadsS;
-      uint32_t zc = 0, cc = 0;
-      // Thread 0 also walks the query and RoPE stages in order and releases
-      // them (the converters' share of their three releases).
-      bool ok = true;
-      auto observe = [&](uint32_t n) {
-        for (uint32_t u = 0; u < n; ++u, ++zc)
-          if (t == 0 && ok) {
-            ok = bwait(ctl, bar(bars->z_full[zc % nz]), (zc / nz) & 1u);
-            if (ok) mbar_arrive(bar(bars->z_empty[zc % nz]));
-          }
-      };
-      each_piece(sv, [&](const Piece& pc) {
-        observe(8);                                // the query stages
-        for (int j = pc.p0; j < pc.p1; j += 2) {
-          observe(1);                              // the RoPE stage
-          for (int c = 0; c < 4; ++c, ++zc, cc += 2) {
-            const uint32_t zs = zc % nz, c0 = cc % NC, c1 = (cc + 1) % NC;
-            if (t == 0 && ok)
-              ok = bwait(ctl, bar(bars->c_empty[c0]), ((cc / NC) & 1u) ^ 1u) &&
-                   bwait(ctl, bar(bars->c_empty[c1]), (((cc + 1) / NC) & 1u) ^ 1u) &&
-                   bwait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u);
-            if (!named_bar_and(kConvBar, kConvThreadsS, ok)) return false;
-            if (t == 0) MLA_TR(6, 1, zc);
-            const uint32_t src = sbase + L::z + zs * kZStage;
-            uint4 in[kCh];
-#pragma unroll
-            for (int u = 0; u < kCh; ++u) {
-              const int o = t + kConvThreadsS * u, r = o >> 3, k = o & 7;
-              if (o < 128 * 8)
-                in[u] = ld_shared_v4(src + uint32_t(r >> 6) * kBox + uint32_t(r & 63) * 128 +
-                                     ((uint32_t(k) ^ uint32_t(r & 7)) << 4));
-            }
-            // every converter has read the stage: the producer may refill it
-            named_bar_sync(kConvBar, kConvThreadsS);
-            if (t == 0) mbar_arrive(bar(bars->z_empty[zs]));
-#pragma unroll
-            for (int u = 0; u < kCh; ++u) {
-              const int o = t + kConvThreadsS * u, r = o >> 3, k = o & 7;
-              if (o >= 128 * 8) continue;
-              // 16 e4m3 values (latent columns 16k..16k+15 of the box) -> fp16
-              // chunks 2(k&3), 2(k&3)+1 of converted stage k >> 2
-              const uint32_t sw = uint32_t(r & 7);
-              const uint32_t dst = sbase + L::c + (k < 4 ? c0 : c1) * kZStage + uint32_t(r >> 6) * kBox +
-                                   uint32_t(r & 63) * 128;
-              const uint32_t ch = uint32_t(2 * (k & 3));
-              st_shared_v4(dst + ((ch ^ sw) << 4), e4m3x2_to_f16x2(in[u].x & 0xFFFFu), e4m3x2_to_f16x2(in[u].x >> 16),
-                           e4m3x2_to_f16x2(in[u].y & 0xFFFFu), e4m3x2_to_f16x2(in[u].y >> 16));
-              st_shared_v4(dst + (((ch + 1u) ^ sw) << 4), e4m3x2_to_f16x2(in[u].z & 0xFFFFu),
-                           e4m3x2_to_f16x2(in[u].z >> 16), e4m3x2_to_f16x2(in[u].w & 0xFFFFu),
-                           e4m3x2_to_f16x2(in[u].w >> 16));
-            }
-            fence_proxy_async_cta();   // the stages feed the tensor core
-            mbar_arrive(bar(bars->c_full[c0]));
-            mbar_arrive(bar(bars->c_full[c1]));
-            if (t == 0) MLA_TR(6, 2, zc);
-          }
-        }
-        return true;
-      });
     } else if (warp >= 4 && warp < 12) {
       // ---- softmax: two warpgroups; thread (h, i) owns row i of the tile
       // (TMEM lane i) for page h of each 2-page block
@@ -806,13 +775,40 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         // 64-127 at +8 KB) is sub-stage c % qbs of stage zc + c / qbs.  BF16
         // cache: boxes 0-8, two per stage, as bf16 pairs in columns [0, 288),
         // group 0 moves boxes 0-4, group 1 boxes 5-8.  FP8 cache: the latent
-        // boxes 0-7, one per stage, as fp16 pairs in columns [0, 256) (the
-        // RoPE box stays in shared memory), 0-3 / 4-7.  Every QK MMA of the
-        // previous piece has completed: its last S was read.
+        // boxes 0-7, one per stage, 0-3 / 4-7, as two e4m3 parts (the RoPE
+        // box stays in shared memory): with a power-of-two scale 2^e per row
+        // that takes the row's largest |value| to at most 448, hi = e4m3(q /
+        // 2^e) keeps 4 of bf16's 8 significant bits and lo = e4m3(q / 2^e -
+        // hi) the rest, exactly (values below 2^-11 of the row's largest
+        // lose at most 2^-19 of it).  hi in columns [0, 128), lo in [128,
+        // 256), four values per column.  Every QK MMA of the previous piece
+        // has completed: its last S was read.
+        float qscale = 1.f;   // FP8 cache: the row's 2^e
         {
           constexpr int nq = kFp8 ? 8 : 9, nq0 = kFp8 ? 4 : 5, qbs = kFp8 ? 1 : 2;
           const uint32_t roff = uint32_t(i >> 6) * kBox + uint32_t(i & 63) * 128;
-          bool big = false;
+          float qinv = 1.f;
+          if constexpr (kFp8) {
+            // the row's largest |value|: each of its two threads reads half
+            // of the latent part from global memory
+            float am = 0.f;
+            if (valid) {
+              const uint16_t* qrow = p.q + (size_t(r) * rows_total + rho) * MLA_D_QK + 256 * h;
+#pragma unroll 4
+              for (int k = 0; k < 32; ++k) {
+                const uint4 w = ld_global_nc_v4(qrow + 8 * k);
+                am = fmaxf(am, fmaxf(fmaxf(bf16_abs_max(w.x), bf16_abs_max(w.y)),
+                                     fmaxf(bf16_abs_max(w.z), bf16_abs_max(w.w))));
+              }
+            }
+            const uint32_t qam = sbase + L::qam;
+            st_shared_u32(qam + 4u * uint32_t(128 * h + i), __float_as_uint(am));
+            named_bar_sync(kSoftmaxBar, kSmThreads);
+            am = fmaxf(am, ld_shared_f32(qam + 4u * uint32_t(128 * (h ^ 1) + i)));
+            const int e = pow2_scale_exp(am);
+            qscale = ldexpf(1.f, e);
+            qinv = ldexpf(1.f, -e);
+          }
 #pragma unroll 1
           for (int c = 0; c < nq; ++c) {
             const uint32_t idx = zc + uint32_t(c / qbs);
@@ -833,13 +829,16 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                 v[4 * k + 3] = x.w;
               }
               if constexpr (kFp8) {
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) v[k] = bf16x2_to_f16x2_checked(v[k], &big);
+                for (int k = 0; k < 16; ++k) split_e4m3x4(v[2 * k], v[2 * k + 1], qinv, &hi[k], &lo[k]);
+                tmem_st16(tmem + lane_off + 16u * c, hi);
+                tmem_st16(tmem + lane_off + kTmemQLo + 16u * c, lo);
+              } else {
+                tmem_st32(tmem + lane_off + 32u * c, v);
               }
-              tmem_st32(tmem + lane_off + 32u * c, v);
             }
           }
-          if (kFp8 && big) flag_status(p.ws, kStatusBadInput);
           if constexpr (kFp8) {
             named_bar_sync(kSoftmaxBar, kSmThreads);
             if (g == 0) mbar_arrive(bar(bars->z_empty[(zc + nq - 1) % nz]));
@@ -870,21 +869,22 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           {
             uint32_t sv0[32], sv1[32];
             if constexpr (kFp8) {
-              // S = scale_j * S_lat + S_rope: the e4m3 values are unscaled
+              // S = 2^e * scale_j * S_lat + S_rope: S_lat is the scaled
+              // query against the unscaled e4m3 values
               tmem_ld32(tmem + lane_off + kTmemSLat + 64u * h, sv0);
               tmem_ld32(tmem + lane_off + kTmemSLat + 64u * h + 32u, sv1);
               tmem_wait_ld();
 #pragma unroll
               for (int c = 0; c < 32; c += 4) {
                 const uint4 s0 = ld_shared_v4(scl + 4u * uint32_t(c)), s1 = ld_shared_v4(scl + 128u + 4u * uint32_t(c));
-                x[c] = __uint_as_float(sv0[c]) * __uint_as_float(s0.x);
-                x[c + 1] = __uint_as_float(sv0[c + 1]) * __uint_as_float(s0.y);
-                x[c + 2] = __uint_as_float(sv0[c + 2]) * __uint_as_float(s0.z);
-                x[c + 3] = __uint_as_float(sv0[c + 3]) * __uint_as_float(s0.w);
-                x[c + 32] = __uint_as_float(sv1[c]) * __uint_as_float(s1.x);
-                x[c + 33] = __uint_as_float(sv1[c + 1]) * __uint_as_float(s1.y);
-                x[c + 34] = __uint_as_float(sv1[c + 2]) * __uint_as_float(s1.z);
-                x[c + 35] = __uint_as_float(sv1[c + 3]) * __uint_as_float(s1.w);
+                x[c] = __uint_as_float(sv0[c]) * (qscale * __uint_as_float(s0.x));
+                x[c + 1] = __uint_as_float(sv0[c + 1]) * (qscale * __uint_as_float(s0.y));
+                x[c + 2] = __uint_as_float(sv0[c + 2]) * (qscale * __uint_as_float(s0.z));
+                x[c + 3] = __uint_as_float(sv0[c + 3]) * (qscale * __uint_as_float(s0.w));
+                x[c + 32] = __uint_as_float(sv1[c]) * (qscale * __uint_as_float(s1.x));
+                x[c + 33] = __uint_as_float(sv1[c + 1]) * (qscale * __uint_as_float(s1.y));
+                x[c + 34] = __uint_as_float(sv1[c + 2]) * (qscale * __uint_as_float(s1.z));
+                x[c + 35] = __uint_as_float(sv1[c + 3]) * (qscale * __uint_as_float(s1.w));
               }
               tmem_ld32(tmem + lane_off + kTmemS + 64u * h, sv0);
               tmem_ld32(tmem + lane_off + kTmemS + 64u * h + 32u, sv1);
