@@ -132,6 +132,28 @@ def test_full_size_configs_sampled(cfg):
 
 # ---- FP8 cache: the kFp8 kernel across the same edge cases ------------------
 
+def test_fp8_query_beyond_fp16_range():
+    """The FP8 kernel's latent scores use a two-part e4m3 copy of the query
+    with a per-row power-of-two scale, so query values far outside fp16's
+    range are as good as any: q * 2^17 with softmax_scale / 2^17 is the same
+    problem (both scalings are exact)."""
+    wl = mw.make(2, 1, 128, [300, 70], cache_dtype="fp8", seed=71, name="fp8_big_query")
+    wl.q = (wl.q.float() * 2.0 ** 17).to(torch.bfloat16)
+    assert float(wl.q.float().abs().max()) > 65504.0
+    wl.softmax_scale = wl.softmax_scale / 2.0 ** 17
+    check_full(wl)
+
+
+def test_fp8_query_rows_of_different_magnitudes():
+    # each head's row scaled by its own power of two, 2^-5 .. 2^2 (larger
+    # logits would test fp32 accumulation, not the split): every row gets
+    # its own scale for the e4m3 split
+    wl = mw.make(2, 1, 128, [500, 129], cache_dtype="fp8", seed=72, name="fp8_row_scales")
+    f = torch.tensor([2.0 ** (j % 8 - 5) for j in range(128)])
+    wl.q = (wl.q.float() * f[None, None, :, None]).to(torch.bfloat16)
+    check_full(wl)
+
+
 def test_fp8_causal_spec_and_packed_tiles():
     check_full(mw.make(3, 16, 128, [200, 16, 700], causal=True, cache_dtype="fp8", seed=13, name="fp8_spec"))
     check_full(mw.make(3, 2, 64, [130, 5, 260], causal=True, cache_dtype="fp8", seed=14, name="fp8_h64s2"))
