@@ -34,6 +34,14 @@ softmax attention over exactly the listed rows, shared by all heads of that
 query token.  Positions outside [0, t_r) (-1 padding) are skipped; a position
 listed twice is two keys.
 
+The split form of the same attention for speculative steps ("MLAvar6+
+Design" on the same page) keeps the o older tokens in latent form and the n
+newest as decompressed per-head keys and values: old token j scores with the
+absorbed query against its cache row and contributes its decompressed value
+row C_j[:512] . W_kvb2[h]^T; new token m scores with the unabsorbed query
+[q_nope | q_pe] against [k_new | its cache row's RoPE part] and contributes
+v_new.  One softmax over both.
+
 The two per-head projections on either side of that attention (same page,
 "Absorption Trick": the key up-projection is folded into the query, and the
 output of the latent attention is decompressed by a separate GEMM) are
@@ -290,3 +298,50 @@ def decompress(o_lat: np.ndarray, w_kvb2: np.ndarray) -> np.ndarray:
     w_kvb2  float64 [h, d, 512]: head j's values are V_j = Z . w_kvb2[j]^T
     Returns float64 [..., h, d]."""
     return np.einsum("...jc,jvc->...jv", o_lat, w_kvb2)
+
+
+def mlavar6_decode(wl, qz: np.ndarray, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,
+                   w_kvb2: np.ndarray, n_new: int):
+    """Split latent + decompressed attention (page "MLA Cost Analysis &
+    Regime Guide", "MLAvar6+ Design"), in float64.
+
+    wl      the workload: cache pool, block table, seqlens, softmax_scale,
+            s_q, causal (its q is not used)
+    qz      [b, s, h, 576] absorbed query (old tokens)
+    q       [b, s, h, d + p] unabsorbed query [q_nope | q_pe] (new tokens)
+    k_new   [b, n, h, d] decompressed keys of each request's n newest tokens
+    v_new   [b, n, h, d] their decompressed values
+    w_kvb2  [h, d, 512] value decompression of the old tokens
+    Token positions: old j < t - n, new m at position t - n + m (m with a
+    negative position, when t < n, does not exist); query i sees positions
+    below visible_len(t, s, i, causal).
+    Returns (out [b, s, h, d], lse [b, s, h])."""
+    b, s, h, _ = qz.shape
+    d = D_HEAD
+    out = np.zeros((b, s, h, d))
+    lse = np.zeros((b, s, h))
+    for r in range(b):
+        t = int(wl.seqlens[r])
+        C = gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale)
+        o = max(t - n_new, 0)
+        for i in range(s):
+            Lv = max(visible_len(t, s, i, wl.causal), 0)
+            jo = min(o, Lv)                                   # visible old tokens
+            ms = np.arange(n_new)
+            pos = t - n_new + ms
+            keep = (pos >= 0) & (pos < Lv)                    # visible new tokens
+            ms, pos = ms[keep], pos[keep]
+            for hh in range(h):
+                x_old = wl.softmax_scale * (C[:jo] @ qz[r, i, hh])
+                x_new = wl.softmax_scale * (k_new[r, ms, hh] @ q[r, i, hh, :d] + C[pos, D_V:] @ q[r, i, hh, d:])
+                x = np.concatenate([x_old, x_new])
+                if x.size == 0:
+                    lse[r, i, hh] = -np.inf
+                    continue
+                m = x.max()
+                z = np.exp(x - m).sum()
+                lse[r, i, hh] = m + math.log(z)
+                w = np.exp(x - lse[r, i, hh])
+                vals = np.concatenate([C[:jo, :D_V] @ w_kvb2[hh].T, v_new[r, ms, hh]])
+                out[r, i, hh] = w @ vals
+    return out, lse

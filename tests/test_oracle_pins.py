@@ -292,6 +292,48 @@ def test_sparse_order_padding_and_duplicates():
     assert np.all(Oz == 0) and np.all(np.isneginf(Lz))
 
 
+# ---- MLAvar6+: old tokens in latent form, the n newest decompressed ---------
+
+def _var6_case(n_new, seed=5):
+    """A causal speculative batch, random per-head projections, and the
+    exact (fp64) decompression of each request's n newest tokens; slots of
+    positions that do not exist (t < n) are NaN."""
+    wl = _tiny([150, 70], h=3, s_q=3, causal=True, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    h = wl.num_heads
+    wk = (torch.randn(h, 512, 128, generator=g, dtype=torch.float64) / math.sqrt(512)).numpy()
+    wv = (torch.randn(h, 128, 512, generator=g, dtype=torch.float64) / math.sqrt(512)).numpy()
+    q = torch.randn(wl.batch, wl.s_q, h, 192, generator=g, dtype=torch.float64).numpy()
+    qz = oracle.absorb(q, wk)
+    k_new = np.full((wl.batch, n_new, h, 128), np.nan)
+    v_new = np.full((wl.batch, n_new, h, 128), np.nan)
+    for r, t in enumerate(wl.seqlens):
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        for m in range(n_new):
+            p = int(t) - n_new + m
+            if p >= 0:
+                k_new[r, m] = np.einsum("c,jcn->jn", C[p, :512], wk)
+                v_new[r, m] = np.einsum("c,jvc->jv", C[p, :512], wv)
+    return wl, wk, wv, q, qz, k_new, v_new
+
+
+@pytest.mark.parametrize("n_new", [0, 1, 3, 64, 100, 150])
+def test_mlavar6_with_exact_decompression_is_the_latent_path(n_new):
+    # whatever n, keeping the newest tokens decompressed changes nothing when
+    # their keys and values are the exact projections of their latent rows;
+    # n = 100 > t = 70 for the second request, n = 150 = t makes the first
+    # request fully decompressed (ordinary MHA)
+    wl, wk, wv, q, qz, k_new, v_new = _var6_case(n_new)
+    out, lse = oracle.mlavar6_decode(wl, qz, q, k_new, v_new, wv, n_new)
+    for r, t in enumerate(wl.seqlens):
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        for i in range(wl.s_q):
+            L = om.visible_len(int(t), wl.s_q, i, True)
+            olat, lref = oracle.attend(qz[r, i], C[:L], wl.softmax_scale)
+            assert np.max(np.abs(out[r, i] - oracle.decompress(olat, wv))) < 1e-12
+            assert np.max(np.abs(lse[r, i] - lref)) < 1e-12
+
+
 def test_uniform_scores_give_mean_of_values():
     # Q = 0: every score is 0, so the weights are 1/L, O is the mean of the
     # value rows and lse = ln L
