@@ -460,6 +460,70 @@ def run_sparse(args, dev, flush, pk):
             "gpu_launches": 4 * args.steps, "cpu_baseline": cpu}
 
 
+def var6_flops(b, h, s, t, n):
+    """The page's MLAvar6+ cost model: 2bhstp + 4bhsnd + 4bhsok (o = t - n)."""
+    return 2 * b * h * s * t * 64 + 4 * b * h * s * n * 128 + 4 * b * h * s * (t - n) * 512
+
+
+def run_var6(args, dev, flush, pk):
+    """MLAvar6+ split decode on the speculative workload (b=32, s=16,
+    t=4096, causal): n = 16 and 64 newest tokens held decompressed, against
+    the latent path with its output decompressed (schedule, decode, combine,
+    decompression), both timed like the decode."""
+    import mla_latent_space_b200 as mla
+    wl = mw.make_config(5, seed=0)
+    b, s, h = wl.batch, wl.s_q, wl.num_heads
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn(b, s, h, 192, generator=g).to(torch.bfloat16).to(dev)
+    wv = mw.make_projections(1, h, seed=8).w_kvb2.to(dev)
+    shape = mla.make_shape(b, s, h, wl.max_pages, wl.num_pages, wl.cache_dtype, wl.causal)
+    qz, pool = wl.q.to(dev), wl.pool.to(dev)
+    bt, sl = torch.from_numpy(wl.block_table).to(dev), torch.from_numpy(wl.seqlens).to(dev)
+    out = torch.empty((b, s, h, 128), dtype=torch.bfloat16, device=dev)
+    lat = torch.empty((b, s, h, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((b, s, h), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, e in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            e.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(e) for a, e in evs) / len(evs) * 1e3
+
+    dec = mla.Decoder(shape, device=dev)
+
+    def latent():
+        dec.schedule(sl)
+        dec.decode(qz, pool, None, bt, sl, wl.softmax_scale, lat, lse)
+        mla.mla_decompress_o(lat, wv, out)
+
+    t_lat = timed(latent)
+    t = int(wl.seqlens[0])
+    res = {"workload": wl.name, "latent_path_us": t_lat,
+           "latent_path_tflops": var6_flops(b, h, s, t, 0) / (t_lat * 1e-6) / 1e12, "split": []}
+    for n in (16, 64):
+        k_new = torch.randn(b, n, h, 128, generator=g).to(torch.bfloat16).to(dev)
+        v_new = torch.randn(b, n, h, 128, generator=g).to(torch.bfloat16).to(dev)
+        vd = mla.Var6Decoder(shape, n, device=dev)
+        us = timed(lambda: vd.decode(qz, q, pool, bt, sl, k_new, v_new, wv, wl.softmax_scale, out, lse))
+        if vd.status() != 0:
+            raise RuntimeError("device status set in the MLAvar6+ timing")
+        res["split"].append({"n_new": n, "us_per_call": us,
+                             "tflops": var6_flops(b, h, s, t, n) / (us * 1e-6) / 1e12})
+    if dec.status() != 0:
+        raise RuntimeError("device status set in the latent-path timing")
+    res["gpu_launches"] = args.steps * (4 + 2 * 6)
+    return res
+
+
 def run_projections_only(args, wl, world, rank):
     """`--projections-only`: the projection timing of run_projections alone,
     on this rank's GPU, printed as its own JSON line."""
@@ -564,6 +628,7 @@ def run_ours(args, wl, world, rank, local):
     proj = None if args.no_projections else run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush,
                                                               peaks()[0])
     sparse = None if args.no_sparse else run_sparse(args, dev, flush, peaks()[0])
+    var6 = None if args.no_var6 else run_var6(args, dev, flush, peaks()[0])
     h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
 
@@ -609,6 +674,8 @@ def run_ours(args, wl, world, rank, local):
         line["mla_attention"] = proj
     if sparse is not None:
         line["sparse_decode"] = sparse
+    if var6 is not None:
+        line["mlavar6"] = var6
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10 s of oracle work: the sample repeated until 10 s have passed
         n_req = max(1, min(wl.batch, args.ref_requests))
@@ -637,6 +704,7 @@ def main():
                     help="time only the query absorption / output decompression kernels and the whole step")
     ap.add_argument("--no-sparse", action="store_true", help="skip the timing of the token-level sparse decode")
     ap.add_argument("--sparse-only", action="store_true", help="time only the token-level sparse decode")
+    ap.add_argument("--no-var6", action="store_true", help="skip the timing of the MLAvar6+ split decode")
     ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
     ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,

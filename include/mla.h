@@ -225,6 +225,38 @@ int mla_sparse_decode_fwd(const mla_shape_t* shape, int topk, const void* q, con
 int mla_sparse_get_device_status(const mla_shape_t* shape, int topk, int num_sms, void* workspace, void* stream,
                                  int* status);
 
+/* ---- MLAvar6+ split attention for speculative steps -------------------------
+ * "MLA Cost Analysis & Regime Guide", section "MLAvar6+ Design": each
+ * request's o = t - n older tokens stay in latent form (the cache), its n
+ * newest are given as decompressed per-head keys and values; one softmax
+ * covers both.  Old token j scores scale * qz . C_j and contributes its
+ * decompressed value C_j[:512] . w_kvb2[head]^T; new token m (position
+ * t - n + m; absent when that is negative) scores scale * (q_nope . k_new[m]
+ * + q_pe . C_{t-n+m}[512:]) and contributes v_new[m].  Query token i sees
+ * positions below t - s_q + i + 1 (causal) or t.  Runs as the latent decode
+ * over the old tokens, the output decompression of its result, and one
+ * kernel that attends over the new tokens and merges by log-sum-exp.
+ *   shape    : as for mla_decode_fwd; s_q <= 32; causal steps need n >= s_q
+ *              (every old token then precedes every query position).
+ *   n_new    : n, 0 <= n <= 2^20 (0: the latent path alone, decompressed).
+ *   qz       : bf16 [batch, s_q, h, 576], the absorbed query (old tokens).
+ *   q        : bf16 [batch, s_q, h, 192] = [q_nope | q_pe] (new tokens).
+ *   kv_cache, kv_scale, block_table, seqlens: as for mla_decode_fwd.
+ *   k_new    : bf16 [batch, n, h, 128] decompressed keys (RoPE part excluded).
+ *   v_new    : bf16 [batch, n, h, 128] decompressed values.
+ *   w_kvb2   : bf16 [h, 128, 512], as for mla_decompress_o.
+ *   workspace: mla_var6_workspace_bytes(shape, n, num_sms of this device)
+ *              bytes, 256-byte aligned, zero-filled before its first use.
+ *   out      : bf16 [batch, s_q, h, 128];  lse: fp32 [batch, s_q, h]. */
+size_t mla_var6_workspace_bytes(const mla_shape_t* shape, int n_new, int num_sms);
+int mla_var6_decode_fwd(const mla_shape_t* shape, int n_new, const void* qz, const void* q, const void* kv_cache,
+                        const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, const void* k_new,
+                        const void* v_new, const void* w_kvb2, float softmax_scale, void* workspace,
+                        size_t workspace_bytes, void* out, float* lse, void* stream);
+/* Device status of the split decode's kernels; as mla_get_device_status. */
+int mla_var6_get_device_status(const mla_shape_t* shape, int n_new, int num_sms, void* workspace, void* stream,
+                               int* status);
+
 /* ---- the projections on either side of the decode -------------------------
  * "MLA Cost Analysis & Regime Guide", section "Absorption Trick": the key
  * up-projection Wk is folded into the query (Q . K^T = (Q . Wk^T) . Z^T),

@@ -78,6 +78,12 @@ def lib() -> ctypes.CDLL:
         L.mla_sparse_decode_fwd.restype = i32
         L.mla_sparse_get_device_status.argtypes = [sp, i32, i32, vp, vp, ctypes.POINTER(i32)]
         L.mla_sparse_get_device_status.restype = i32
+        L.mla_var6_workspace_bytes.argtypes = [sp, i32, i32]
+        L.mla_var6_workspace_bytes.restype = sz
+        L.mla_var6_decode_fwd.argtypes = [sp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp, sz, vp, vp, vp]
+        L.mla_var6_decode_fwd.restype = i32
+        L.mla_var6_get_device_status.argtypes = [sp, i32, i32, vp, vp, ctypes.POINTER(i32)]
+        L.mla_var6_get_device_status.restype = i32
         L.mla_absorb_q.argtypes = [i32, i32, vp, vp, vp, vp, vp]
         L.mla_absorb_q.restype = i32
         L.mla_decompress_o.argtypes = [i32, i32, vp, vp, vp, vp, vp]
@@ -169,8 +175,10 @@ def _check_decode_tensors(shape, q, kv_cache, kv_scale, block_table, seqlens, ou
         _need(kv_scale, "kv_scale", torch.float32, (shape.num_pages, PAGE))
     _need(block_table, "block_table", torch.int32, (b, shape.max_pages_per_seq))
     _need(seqlens, "seqlens", torch.int32, (b,))
-    _need(out, "out", torch.bfloat16, (b, s, h, D_V))
-    _need(lse, "lse", torch.float32, (b, s, h))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, (b, s, h, D_V))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (b, s, h))
 
 
 def _decode_common(fn, where, shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched,
@@ -269,6 +277,44 @@ class SparseDecoder:
         _check(lib().mla_sparse_get_device_status(ctypes.byref(self.shape), self.topk, self.n_sms,
                                                   _ptr(self.workspace), _stream(stream), ctypes.byref(st)),
                "mla_sparse_get_device_status")
+        return int(st.value)
+
+
+class Var6Decoder:
+    """MLAvar6+ split decode through the C ABI: the older tokens in latent
+    form, the n newest as decompressed per-head keys and values.  Holds the
+    zero-filled workspace for one shape, n and device."""
+
+    def __init__(self, shape: mla_shape_t, n_new: int, device=None):
+        self.shape, self.n_new = shape, int(n_new)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.n_sms = num_sms(self.device)
+        nb = int(lib().mla_var6_workspace_bytes(ctypes.byref(shape), self.n_new, self.n_sms))
+        if nb == 0:
+            raise MLAError(-2, "Var6Decoder: shape not supported (s_q <= 32; causal steps need n >= s_q)")
+        self.workspace = torch.zeros(nb, dtype=torch.uint8, device=self.device)
+
+    def decode(self, qz, q, kv_cache, block_table, seqlens, k_new, v_new, w_kvb2, softmax_scale, out, lse,
+               stream=None, kv_scale=None):
+        sh, n = self.shape, self.n_new
+        _check_decode_tensors(sh, qz, kv_cache, kv_scale, block_table, seqlens, None, None)
+        _need(q, "q", torch.bfloat16, (sh.batch, sh.s_q, sh.num_heads, D_HEAD + D_ROPE))
+        _need(k_new, "k_new", torch.bfloat16, (sh.batch, n, sh.num_heads, D_HEAD))
+        _need(v_new, "v_new", torch.bfloat16, (sh.batch, n, sh.num_heads, D_HEAD))
+        _need(w_kvb2, "w_kvb2", torch.bfloat16, (sh.num_heads, D_HEAD, D_V))
+        _need(out, "out", torch.bfloat16, (sh.batch, sh.s_q, sh.num_heads, D_HEAD))
+        _need(lse, "lse", torch.float32, (sh.batch, sh.s_q, sh.num_heads))
+        rc = lib().mla_var6_decode_fwd(ctypes.byref(sh), n, _ptr(qz), _ptr(q), _ptr(kv_cache), _ptr(kv_scale),
+                                       _ptr(block_table), _ptr(seqlens), _ptr(k_new), _ptr(v_new), _ptr(w_kvb2),
+                                       float(softmax_scale), _ptr(self.workspace), self.workspace.numel(), _ptr(out),
+                                       _ptr(lse), _stream(stream))
+        _check(rc, "mla_var6_decode_fwd")
+
+    def status(self, stream=None) -> int:
+        st = ctypes.c_int(0)
+        _check(lib().mla_var6_get_device_status(ctypes.byref(self.shape), self.n_new, self.n_sms,
+                                                _ptr(self.workspace), _stream(stream), ctypes.byref(st)),
+               "mla_var6_get_device_status")
         return int(st.value)
 
 

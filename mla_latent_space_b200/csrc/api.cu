@@ -25,6 +25,13 @@ cudaError_t launch_sparse_gather(const int32_t* indices, int topk, const int32_t
                                  const int32_t* block_table, int max_pages, int num_pages, const void* pool,
                                  const float* kv_scale, void* scratch, float* vscale, int vpages, int32_t* vseqlens,
                                  int32_t* vbt, void* status_ws, bool fp8, cudaStream_t stream);
+cudaError_t launch_var6_old_len(const int32_t* seqlens, int batch, int n_new, int max_pages, int32_t* old_len,
+                                cudaStream_t stream);
+cudaError_t launch_var6_new(const void* q, const void* k_new, const void* v_new, const void* pool, bool fp8,
+                            const int32_t* block_table, const int32_t* seqlens, const void* o_old,
+                            const float* lse_old, int batch, int s_q, int heads, int n_new, int max_pages,
+                            int num_pages, int causal, float scale, void* out, float* lse, void* status_ws,
+                            cudaStream_t stream);
 int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* qz, int32_t* status,
                     cudaStream_t stream);
 int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
@@ -152,6 +159,42 @@ bool sparse_layout(const mla_shape_t* s, int topk, int num_sms, SparseLayout* L)
   off = up(off + size_t(V) * size_t(vpages) * page_bytes);
   L->vscale = off;
   if (fp8) off = up(off + size_t(V) * size_t(vpages) * MLA_PAGE_SIZE * 4);
+  L->total = off;
+  return true;
+}
+
+// Workspace of the MLAvar6+ split decode (every region 256-byte aligned):
+// the old lengths t - n, the schedule and decode workspace of the latent
+// part (a non-causal decode over the old tokens), its latent output and
+// lse, and its decompressed output.
+struct Var6Layout {
+  mla_shape_t oshape;
+  size_t oldlen, sched, sched_bytes, ws, ws_bytes, olat, lse_old, oold, total;
+};
+
+bool var6_layout(const mla_shape_t* s, int n_new, int num_sms, Var6Layout* L) {
+  if (check_shape(s) != MLA_OK || num_sms < 1 || n_new < 0 || n_new > (1 << 20)) return false;
+  if (s->s_q > 32 || s->num_heads > 65535) return false;
+  if (s->causal && n_new < s->s_q) return false;   // every old token must be visible to every query row
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  L->oshape = *s;
+  L->oshape.causal = 0;
+  const size_t rows = size_t(s->batch) * s->s_q * s->num_heads;
+  size_t off = 0;
+  L->oldlen = off;
+  off = up(off + 4 * size_t(s->batch));
+  L->sched = off;
+  L->sched_bytes = sched_bytes_for(&L->oshape, num_sms);
+  off = up(off + L->sched_bytes);
+  L->ws = off;
+  L->ws_bytes = kStatusBytes + size_t(max_slots_for(num_workers_for(num_sms))) * kSlotBytes;
+  off = up(off + L->ws_bytes);
+  L->olat = off;
+  off = up(off + rows * MLA_D_V * 2);
+  L->lse_old = off;
+  off = up(off + rows * 4);
+  L->oold = off;
+  off = up(off + rows * MLA_D_HEAD * 2);
   L->total = off;
   return true;
 }
@@ -302,6 +345,70 @@ int mla_sparse_get_device_status(const mla_shape_t* shape, int topk, int num_sms
                                  int* status) {
   SparseLayout L;
   if (!workspace || !status || !sparse_layout(shape, topk, num_sms, &L)) return MLA_ERR_INVALID_ARG;
+  char* w = static_cast<char*>(workspace);
+  return mla_get_device_status(w + L.sched, w + L.ws, stream, status);
+}
+
+size_t mla_var6_workspace_bytes(const mla_shape_t* shape, int n_new, int num_sms) {
+  Var6Layout L;
+  return var6_layout(shape, n_new, num_sms, &L) ? L.total : 0;
+}
+
+int mla_var6_decode_fwd(const mla_shape_t* shape, int n_new, const void* qz, const void* q, const void* kv_cache,
+                        const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, const void* k_new,
+                        const void* v_new, const void* w_kvb2, float softmax_scale, void* workspace,
+                        size_t workspace_bytes, void* out, float* lse, void* stream) {
+  int rc = check_shape(shape);
+  if (rc != MLA_OK) return rc;
+  const bool fp8 = shape->cache_dtype == MLA_CACHE_FP8_E4M3;
+  if (n_new < 0 || n_new > (1 << 20) || (shape->causal && n_new < shape->s_q)) return MLA_ERR_INVALID_ARG;
+  if (shape->s_q > 32 || shape->num_heads > 65535) return MLA_ERR_UNSUPPORTED;
+  if (!qz || !q || !kv_cache || !block_table || !seqlens || !w_kvb2 || !workspace || !out || !lse)
+    return MLA_ERR_INVALID_ARG;
+  if (n_new > 0 && (!k_new || !v_new)) return MLA_ERR_INVALID_ARG;
+  if (fp8 && !kv_scale) return MLA_ERR_INVALID_ARG;
+  if (!aligned(qz, 16) || !aligned(q, 16) || !aligned(kv_cache, 256) || !aligned(block_table, 4) ||
+      !aligned(seqlens, 4) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(w_kvb2, 16) ||
+      !aligned(workspace, 256) || !aligned(out, 16) || !aligned(lse, 4) || (kv_scale && !aligned(kv_scale, 4)))
+    return MLA_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((rc = device_sms(&sms)) != MLA_OK) return rc;
+  Var6Layout L;
+  if (!var6_layout(shape, n_new, sms, &L)) return MLA_ERR_UNSUPPORTED;
+  if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE;
+  char* w = static_cast<char*>(workspace);
+  int32_t* oldlen = reinterpret_cast<int32_t*>(w + L.oldlen);
+  void* sched = w + L.sched;
+  void* ws = w + L.ws;
+  void* olat = w + L.olat;
+  float* lse_old = reinterpret_cast<float*>(w + L.lse_old);
+  void* oold = w + L.oold;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int b = shape->batch, s = shape->s_q, h = shape->num_heads;
+  if (launch_var6_old_len(seqlens, b, n_new, shape->max_pages_per_seq, oldlen, st) != cudaSuccess) return MLA_ERR_CUDA;
+  const ShapeInfo si = shape_info(&L.oshape);
+  if (launch_schedule(oldlen, si, num_workers_for(sms), static_cast<int32_t*>(sched), st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const int cap = cap_slots_for(L.ws_bytes);
+  rc = launch_decode_sm100(&L.oshape, qz, kv_cache, kv_scale, block_table, oldlen, softmax_scale, sched, ws, cap, olat,
+                           lse_old, st);
+  if (rc != MLA_OK) return rc;
+  if (launch_combine(sched, ws, olat, lse_old, si.batch * si.tiles_per_req, cap, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  rc = launch_decompress_o(b * s, h, olat, w_kvb2, oold, static_cast<int32_t*>(ws), st);
+  if (rc != MLA_OK) return rc;
+  return launch_var6_new(q, k_new, v_new, kv_cache, fp8, block_table, seqlens, oold, lse_old, b, s, h, n_new,
+                         shape->max_pages_per_seq, shape->num_pages, shape->causal, softmax_scale, out, lse, ws,
+                         st) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+int mla_var6_get_device_status(const mla_shape_t* shape, int n_new, int num_sms, void* workspace, void* stream,
+                               int* status) {
+  Var6Layout L;
+  if (!workspace || !status || !var6_layout(shape, n_new, num_sms, &L)) return MLA_ERR_INVALID_ARG;
   char* w = static_cast<char*>(workspace);
   return mla_get_device_status(w + L.sched, w + L.ws, stream, status);
 }

@@ -300,6 +300,35 @@ def decompress(o_lat: np.ndarray, w_kvb2: np.ndarray) -> np.ndarray:
     return np.einsum("...jc,jvc->...jv", o_lat, w_kvb2)
 
 
+def new_token_attention(wl, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray, n_new: int):
+    """Attention of every query row over the n decompressed newest tokens
+    alone (the second part of the split form): keys [k_new | the cache
+    row's RoPE part], values v_new, the same positions and visibility as
+    mlavar6_decode.  Returns (o [b, s, h, d], lse [b, s, h]); a row that
+    sees none of them gives o = 0, lse = -inf."""
+    b, s, h, _ = q.shape
+    d = D_HEAD
+    out = np.zeros((b, s, h, d))
+    lse = np.full((b, s, h), -np.inf)
+    for r in range(b):
+        t = int(wl.seqlens[r])
+        C = gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale)
+        for i in range(s):
+            Lv = max(visible_len(t, s, i, wl.causal), 0)
+            ms = np.arange(n_new)
+            pos = t - n_new + ms
+            keep = (pos >= 0) & (pos < Lv)
+            ms, pos = ms[keep], pos[keep]
+            if ms.size == 0:
+                continue
+            for hh in range(h):
+                x = wl.softmax_scale * (k_new[r, ms, hh] @ q[r, i, hh, :d] + C[pos, D_V:] @ q[r, i, hh, d:])
+                m = x.max()
+                lse[r, i, hh] = m + math.log(np.exp(x - m).sum())
+                out[r, i, hh] = np.exp(x - lse[r, i, hh]) @ v_new[r, ms, hh]
+    return out, lse
+
+
 def mlavar6_decode(wl, qz: np.ndarray, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,
                    w_kvb2: np.ndarray, n_new: int):
     """Split latent + decompressed attention (page "MLA Cost Analysis &

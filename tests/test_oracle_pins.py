@@ -334,6 +334,27 @@ def test_mlavar6_with_exact_decompression_is_the_latent_path(n_new):
             assert np.max(np.abs(lse[r, i] - lref)) < 1e-12
 
 
+@pytest.mark.parametrize("n_new", [3, 64, 100])
+def test_mlavar6_is_the_merge_of_its_two_parts(n_new):
+    # the joint softmax over old and new tokens equals the log-sum-exp merge
+    # of the decompressed latent attention over the old tokens and the
+    # attention over the new ones (arbitrary k_new / v_new: the identity
+    # does not depend on them being projections)
+    wl, wk, wv, q, qz, _, _ = _var6_case(n_new, seed=9)
+    g = np.random.default_rng(3)
+    k_new = g.standard_normal((wl.batch, n_new, wl.num_heads, 128))
+    v_new = g.standard_normal((wl.batch, n_new, wl.num_heads, 128))
+    out, lse = oracle.mlavar6_decode(wl, qz, q, k_new, v_new, wv, n_new)
+    o_new, l_new = oracle.new_token_attention(wl, q, k_new, v_new, n_new)
+    for r, t in enumerate(wl.seqlens):
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        old = max(int(t) - n_new, 0)
+        for i in range(wl.s_q):
+            olat, l_old = oracle.attend(qz[r, i], C[:old], wl.softmax_scale)
+            o, L = oracle.combine([(oracle.decompress(olat, wv), l_old), (o_new[r, i], l_new[r, i])])
+            assert np.max(np.abs(out[r, i] - o)) < 1e-12 and np.max(np.abs(lse[r, i] - L)) < 1e-12
+
+
 def test_uniform_scores_give_mean_of_values():
     # Q = 0: every score is 0, so the weights are 1/L, O is the mean of the
     # value rows and lse = ln L
