@@ -37,6 +37,13 @@
 // 1e-3 of relative L1 error in O; fp16 keeps it near 2e-4.  The MMA needs
 // both operands of one type, hence the fp16 copy of V.
 //
+// FP8 cache (kFp8): the score CTA's ring carries the cache's e4m3 latent
+// columns as they are, and the latent scores run as kind::f8f6f4 MMAs
+// against a two-part e4m3 copy of the query (hi + lo with a per-row
+// power-of-two scale, which reproduces the bf16 query); the RoPE part
+// stays a bf16 MMA.  The output CTA expands each page's e4m3 values, times
+// their per-token scales, to fp16 in place.
+//
 // Every wait is bounded: a wait that runs out sets a status bit in the
 // workspace, tells the peer CTA to stop, and the kernel drains its
 // in-flight copies and MMAs, frees TMEM and returns.
@@ -181,8 +188,8 @@ struct Params {
 // role of cluster 0 records (event << 24 | index, clock64, 0) into
 // trace[role][2048][3]; the last entry of roles 6 and 7 holds one
 // (0, clock64, %globaltimer) pair per CTA taken right after the start-up
-// cluster barrier, to line the two SMs' clocks up (role 6 also records the
-// score CTA's FP8 converters).  Only the SM clock is read per event (the global timer
+// cluster barrier, to line the two SMs' clocks up.  Only the SM clock is
+// read per event (the global timer
 // is far slower to read and would distort the timeline).  In normal builds
 // the hooks compile to nothing.
 #ifdef MLA_TRACE
