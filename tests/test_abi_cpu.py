@@ -127,6 +127,27 @@ def test_sparse_workspace_and_argument_checks():
     assert L.mla_sparse_decode_fwd(*args(mla.make_shape(4, 2, 128, 8, 64, causal=True), 64)) == -1
 
 
+def test_var6_workspace_and_argument_checks():
+    L = mla.lib()
+    s = mla.make_shape(32, 16, 128, 64, 2048, causal=True)
+    # old lengths, schedule, decode workspace, then the latent output (bf16 x 512), its lse (fp32) and its
+    # decompression (bf16 x 128) for 32 x 16 x 128 rows
+    rows = 32 * 16 * 128
+    nb = L.mla_var6_workspace_bytes(ctypes.byref(s), 64, 148)
+    assert rows * (1024 + 4 + 256) < nb < rows * (1024 + 4 + 256) + (64 << 20)
+    assert L.mla_var6_workspace_bytes(ctypes.byref(s), 8, 148) == 0          # causal needs n >= s_q
+    assert L.mla_var6_workspace_bytes(ctypes.byref(mla.make_shape(32, 16, 128, 64, 2048)), 8, 148) > 0
+    assert L.mla_var6_workspace_bytes(ctypes.byref(mla.make_shape(2, 33, 128, 64, 2048)), 64, 148) == 0
+    assert L.mla_var6_workspace_bytes(ctypes.byref(s), -1, 148) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    args = lambda sh, n, kn=fake, qz=fake: (ctypes.byref(sh), n, qz, fake, fake, None, fake, fake, kn, fake, fake,
+                                            0.1, fake, 1 << 40, fake, fake, None)
+    assert L.mla_var6_decode_fwd(*args(s, 8)) == -1                            # causal, n < s_q
+    assert L.mla_var6_decode_fwd(*args(s, 64, kn=None)) == -1                  # n > 0 needs k_new
+    assert L.mla_var6_decode_fwd(*args(s, 64, qz=ctypes.c_void_p((1 << 20) + 8))) == -1
+    assert L.mla_var6_decode_fwd(*args(mla.make_shape(2, 33, 128, 64, 2048), 64)) == -2
+
+
 def test_projections_reject_bad_args_before_any_launch():
     L = mla.lib()
     fake = ctypes.c_void_p(1 << 20)
