@@ -7,13 +7,17 @@
  * every head scores directly against the shared latent cache,
  *
  *     S = scale * Qz . C^T            C = cache rows [latent 512 | RoPE 64]
- *     O = softmax(S) . C[:, :512]     (decompression O . W_v^T is left to a
- *                                      separate GEMM, outside this library)
+ *     O = softmax(S) . C[:, :512]     (decompressed by a separate GEMM)
  *
  * Shapes follow the page's "Tensor Shapes" table (h=128, k=512, p=64).  The
  * split-KV scheduler and the log-sum-exp merge of partial results follow the
  * FlashMLA-2 newsletter page ("Architectural Analysis": sequence partitions
  * balanced across SMs for jagged batches).
+ *
+ * Around the decode: the query absorption and the output decompression
+ * (mla_absorb_q, mla_decompress_o), token-level sparse decode over listed
+ * cache positions (mla_sparse_*), and the MLAvar6+ split decode with the
+ * newest tokens held decompressed (mla_var6_*).
  *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The
