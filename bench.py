@@ -625,10 +625,13 @@ def run_ours(args, wl, world, rank, local):
     # wait for its upload; a buffer is reused only after the step that last
     # used it has been downloaded).  The cache (302 MB) is larger than L2.
     e2e_ms = run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world)
-    proj = None if args.no_projections else run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush,
-                                                              peaks()[0])
-    sparse = None if args.no_sparse else run_sparse(args, dev, flush, peaks()[0])
-    var6 = None if args.no_var6 else run_var6(args, dev, flush, peaks()[0])
+    # the extras (the rows around the decode) are timed in single-GPU runs; a
+    # multi-GPU run measures the headline step on every replica
+    extras = world == 1
+    proj = run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, peaks()[0]) \
+        if extras and not args.no_projections else None
+    sparse = run_sparse(args, dev, flush, peaks()[0]) if extras and not args.no_sparse else None
+    var6 = run_var6(args, dev, flush, peaks()[0]) if extras and not args.no_var6 else None
     h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
 
