@@ -237,8 +237,9 @@ def _rows_as_workload(wl, r, i, pos):
                        pool=pool, kv_scale=None, softmax_scale=wl.softmax_scale)
 
 
-def test_sparse_with_every_position_is_the_dense_decode():
-    wl = _tiny([70, 130, 5], h=3, s_q=2)
+@pytest.mark.parametrize("cache_dtype", ["bf16", "fp8"])
+def test_sparse_with_every_position_is_the_dense_decode(cache_dtype):
+    wl = _tiny([70, 130, 5], h=3, s_q=2, cache_dtype=cache_dtype)
     idx = np.full((3, 2, 140), -1, dtype=np.int32)
     for r, t in enumerate(wl.seqlens):
         idx[r, :, :t] = np.arange(t)
@@ -294,11 +295,11 @@ def test_sparse_order_padding_and_duplicates():
 
 # ---- MLAvar6+: old tokens in latent form, the n newest decompressed ---------
 
-def _var6_case(n_new, seed=5):
+def _var6_case(n_new, seed=5, cache_dtype="bf16"):
     """A causal speculative batch, random per-head projections, and the
     exact (fp64) decompression of each request's n newest tokens; slots of
     positions that do not exist (t < n) are NaN."""
-    wl = _tiny([150, 70], h=3, s_q=3, causal=True, seed=seed)
+    wl = _tiny([150, 70], h=3, s_q=3, causal=True, seed=seed, cache_dtype=cache_dtype)
     g = torch.Generator().manual_seed(seed + 1)
     h = wl.num_heads
     wk = (torch.randn(h, 512, 128, generator=g, dtype=torch.float64) / math.sqrt(512)).numpy()
@@ -308,7 +309,7 @@ def _var6_case(n_new, seed=5):
     k_new = np.full((wl.batch, n_new, h, 128), np.nan)
     v_new = np.full((wl.batch, n_new, h, 128), np.nan)
     for r, t in enumerate(wl.seqlens):
-        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t), wl.kv_scale)
         for m in range(n_new):
             p = int(t) - n_new + m
             if p >= 0:
@@ -317,16 +318,17 @@ def _var6_case(n_new, seed=5):
     return wl, wk, wv, q, qz, k_new, v_new
 
 
-@pytest.mark.parametrize("n_new", [0, 1, 3, 64, 100, 150])
-def test_mlavar6_with_exact_decompression_is_the_latent_path(n_new):
+@pytest.mark.parametrize("n_new,cache_dtype", [(0, "bf16"), (1, "bf16"), (3, "bf16"), (64, "bf16"),
+                                               (100, "bf16"), (150, "bf16"), (64, "fp8")])
+def test_mlavar6_with_exact_decompression_is_the_latent_path(n_new, cache_dtype):
     # whatever n, keeping the newest tokens decompressed changes nothing when
     # their keys and values are the exact projections of their latent rows;
     # n = 100 > t = 70 for the second request, n = 150 = t makes the first
     # request fully decompressed (ordinary MHA)
-    wl, wk, wv, q, qz, k_new, v_new = _var6_case(n_new)
+    wl, wk, wv, q, qz, k_new, v_new = _var6_case(n_new, cache_dtype=cache_dtype)
     out, lse = oracle.mlavar6_decode(wl, qz, q, k_new, v_new, wv, n_new)
     for r, t in enumerate(wl.seqlens):
-        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t), wl.kv_scale)
         for i in range(wl.s_q):
             L = om.visible_len(int(t), wl.s_q, i, True)
             olat, lref = oracle.attend(qz[r, i], C[:L], wl.softmax_scale)
@@ -347,7 +349,7 @@ def test_mlavar6_is_the_merge_of_its_two_parts(n_new):
     out, lse = oracle.mlavar6_decode(wl, qz, q, k_new, v_new, wv, n_new)
     o_new, l_new = oracle.new_token_attention(wl, q, k_new, v_new, n_new)
     for r, t in enumerate(wl.seqlens):
-        C = om.gather_rows(wl.pool, wl.block_table, r, int(t))
+        C = om.gather_rows(wl.pool, wl.block_table, r, int(t), wl.kv_scale)
         old = max(int(t) - n_new, 0)
         for i in range(wl.s_q):
             olat, l_old = oracle.attend(qz[r, i], C[:old], wl.softmax_scale)
