@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 256 << 20
 # were taken on: reported as null as soon as any of them differs (checked by
 # content hash at run time).
 TRAFFIC_SOURCES_SHA1 = {
-    "mla_latent_space_b200/csrc/decode_sm100.cu": "7ac2bdb1034fc09929672aeaa1ce5dc3be762615",
+    "mla_latent_space_b200/csrc/decode_sm100.cu": "4fcb6e9d788f6c4d667bf4245664a7b4df75dc8b",
     "mla_latent_space_b200/csrc/sm100_ptx.cuh": "a666c6fb95adecc45850f281b1be3ecacba5d16c",
     "mla_latent_space_b200/csrc/kernel_util.cuh": "c304dedb0965e65632e557168f97693bf2077cdb",
     "mla_latent_space_b200/csrc/common.cuh": "1bda35f3e244dc99d70c2901283243f600e444f6",

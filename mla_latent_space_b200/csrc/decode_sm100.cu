@@ -361,14 +361,19 @@ __device__ __forceinline__ float bf16_abs_max(uint32_t w) {
   return fmaxf(fabsf(__uint_as_float(w << 16)), fabsf(__uint_as_float(w & 0xFFFF0000u)));
 }
 
-// e with am / 2^e <= 448 (e4m3's largest finite value), smallest such; 0
-// for am = 0 or a non-finite am (its NaN or infinity then reaches S as is).
+// e with am / 2^e <= 448 (e4m3's largest finite value), the smallest such
+// but at least -126, so that 2^-e stays finite (a row that small loses
+// nothing that matters: its values still land in e4m3's range); 0 for
+// am = 0 or a non-finite am (its NaN or infinity then reaches S as is).
+// frexpf gives the estimate; the loops correct it by at most a few steps
+// (at most 126 for a subnormal am) and always end.
 __device__ __forceinline__ int pow2_scale_exp(float am) {
   if (!(am > 0.f) || !(am <= 3.402823466e38f)) return 0;
-  int e = int(ceilf(log2f(am * (1.f / 448.f))));
-  while (ldexpf(am, -e) > 448.f) ++e;        // log2f's rounding, either way
-  while (ldexpf(am, -(e - 1)) <= 448.f) --e;
-  return e;
+  int e = 0;
+  frexpf(am * (1.f / 448.f), &e);   // am / 448 = m 2^e, 0.5 <= m < 1
+  while (ldexpf(am, -e) > 448.f) ++e;
+  while (e > -126 && ldexpf(am, -(e - 1)) <= 448.f) --e;
+  return e < -126 ? -126 : e;
 }
 
 // Four bf16 values (w01, w23, low half first) times `inv` (a power of two)

@@ -144,6 +144,16 @@ def test_fp8_query_beyond_fp16_range():
     check_full(wl)
 
 
+def test_fp8_query_far_below_normal_range():
+    """The other end: q * 2^-122 with softmax_scale * 2^122.  The row's
+    power-of-two scale would be 2^-128; it is held at 2^-126 so that its
+    inverse stays finite, and the e4m3 split still covers the row."""
+    wl = mw.make(2, 1, 128, [300, 70], cache_dtype="fp8", seed=73, name="fp8_tiny_query")
+    wl.q = (wl.q.float() * 2.0 ** -122).to(torch.bfloat16)
+    wl.softmax_scale = wl.softmax_scale * 2.0 ** 122
+    check_full(wl)
+
+
 def test_fp8_query_rows_of_different_magnitudes():
     # each head's row scaled by its own power of two, 2^-5 .. 2^2 (larger
     # logits would test fp32 accumulation, not the split): every row gets
