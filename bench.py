@@ -37,17 +37,17 @@ from mla_workloads import cost  # noqa: E402
 
 METRIC = "MLA decode TFLOPS & KV GB/s vs B200 roofline (h=128,k=512,p=64,t=4096)"
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) of one decode launch per workload, from the ncu
-# captures summarised in profiles/.  Valid only for the kernel sources they
-# were taken on: reported as null as soon as any of them differs (checked by
-# content hash at run time).
+# DRAM bytes (read + write) of one decode launch per workload, from one ncu
+# capture of dram__bytes_read.sum + dram__bytes_write.sum each.  Valid only
+# for the kernel sources they were taken on: reported as null as soon as any
+# of them differs (checked by content hash at run time).
 TRAFFIC_SOURCES_SHA1 = {
     "mla_latent_space_b200/csrc/decode_sm100.cu": "4fcb6e9d788f6c4d667bf4245664a7b4df75dc8b",
     "mla_latent_space_b200/csrc/sm100_ptx.cuh": "a666c6fb95adecc45850f281b1be3ecacba5d16c",
     "mla_latent_space_b200/csrc/kernel_util.cuh": "c304dedb0965e65632e557168f97693bf2077cdb",
     "mla_latent_space_b200/csrc/common.cuh": "1bda35f3e244dc99d70c2901283243f600e444f6",
 }
-TRAFFIC_BYTES = {   # profiles/decode_sm100_dsv3_b64_h128_t4096.md, profiles/decode_sm100_fp8_b64_h128_t32768.md
+TRAFFIC_BYTES = {
     "dsv3_b64_h128_t4096_paged": 311.547136e6 + 4.920576e6,
     "fp8_b64_h128_t32768": 1374.59968e6 + 23.452416e6,
 }
@@ -82,51 +82,75 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """SM clock, power and clock-event reasons of this process's GPU, sampled
+    every 10 ms through NVML on a background thread while the timed region
+    runs (nvidia-smi's own loop is too coarse for a region of a second)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
+               ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.cuda_index, self.period = cuda_index, period_s
+        self.samples, self.reasons, self.power = [], set(), []
+        self.max_mhz, self.err = None, None
+        self._stop, self._thread, self._nvml = None, None, None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        try:   # match the CUDA device by UUID (CUDA and NVML may number GPUs differently)
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
-                                          "-i", str(self.index), "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            h = self._handle()
+            nv = self._nvml
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            bits = {}
+            for name, suffix in self.REASONS:
+                v = getattr(nv, "nvmlClocksEventReason" + suffix, getattr(nv, "nvmlClocksThrottleReason" + suffix, 0))
+                bits[name] = int(v)
+        except Exception as e:   # no NVML: the line says so
+            self.err = f"nvml unavailable: {type(e).__name__}"
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
+                    r = int(get_reasons(h)) if get_reasons else 0
+                    for name, bit in bits.items():
+                        if bit and r & bit:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "not sampled"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=5)
         try:
-            out = self.proc.communicate(timeout=5)[0]
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out = self.proc.communicate()[0]
-        sms, mx, reasons, power = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sms.append(float(f[1]))
-                mx = float(f[2])
-                power.append(float(f[3]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sms),
-                "power_w_max": max(power) if power else None}
+            self._nvml.nvmlShutdown()
+        except Exception:
+            pass
+        sm = self.samples
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(sm),
+                "power_w_max": max(self.power) if self.power else None, "source": "nvml, 10 ms"}
 
 
 def dist_setup(n_gpus):
@@ -172,37 +196,26 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_sample(wl, n_req):
-    """Times the fp64 oracle on the first n_req requests; returns
-    (seconds, flops of the sample, description)."""
-    import oracle
-    rows = [(r, i) for r in range(n_req) for i in range(wl.s_q)]
-    t0 = time.perf_counter()
-    oracle.decode(wl, rows=rows)
-    dt = time.perf_counter() - t0
-    st = int(wl.seqlens[:n_req].astype(np.int64).sum())
-    fl = cost.mla_flops(n_req, wl.num_heads, wl.s_q, None, sum_t=st)
-    return dt, fl, f"{n_req} of {wl.batch} requests ({st} cached tokens, all {wl.num_heads} heads)"
-
-
 def run_reference(args, wl, world, rank):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the host
+    cores; each step is a bounded sample of the workload (whole requests in
+    batch order until `--ref-seconds` have passed)."""
     if rank != 0:
         return
-    n_req = max(1, min(wl.batch, args.ref_requests))
-    for _ in range(min(args.warmup, 1)):
-        oracle_sample(wl, 1)   # warm the BLAS threads (untimed)
-    times, fl, desc = [], 0.0, ""
+    import oracle
+    oracle.decode(wl, rows=[(0, 0)])   # warm the BLAS threads (untimed)
+    rates, secs, desc = [], [], ""
+    budget = min(args.ref_seconds, 120.0 / max(1, args.steps))   # the whole run within about two minutes
     for _ in range(args.steps):
-        dt, fl, desc = oracle_sample(wl, n_req)
-        times.append(dt)
-    sec = sum(times) / len(times)
-    tflops = fl / sec / 1e12
+        tf, sec, desc = oracle_timed(wl, budget)
+        rates.append(tf)
+        secs.append(sec)
+    tflops = sum(rates) / len(rates)
     cores = blas_threads()
     line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.num_heads,
-                       "seq_len": int(wl.seqlens.max()), "sample": desc},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(secs) / len(secs) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(wl, world),
             "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
             "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -272,7 +285,7 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
         st = dd.status()
         if st != 0:
             raise RuntimeError(f"device status in the end-to-end loop: {mla.error_string(st)}")
-    K = args.steps
+    K = extra_steps(args)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -284,6 +297,12 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
     torch.cuda.synchronize()
     barrier(world)
     return max_over_ranks(t0.elapsed_time(t1) / K, world)
+
+
+def extra_steps(args):
+    """Timed launches of each secondary measurement (projections, sparse,
+    MLAvar6+, the end-to-end loop): the headline's K, at most 100."""
+    return max(1, min(args.steps, 100))
 
 
 def proj_bytes(rows, heads):
@@ -329,7 +348,7 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
         for _ in range(args.warmup):
             flush.zero_()
             fn()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(extra_steps(args))]
         torch.cuda.synchronize()
         for a, b in evs:
             flush.zero_()
@@ -389,7 +408,7 @@ def run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, pk):
         res["cpu_baseline"] = {"kind": "oracle", "cores": blas_threads(), "absorb_us": (t1 - t0) * 1e6,
                                "decompress_us": (t2 - t1) * 1e6, "sample": f"all {R} rows x {h} heads"}
     # timed launches: absorb alone, decompress alone, and the chain's five kernels (twice: launched, replayed)
-    res["gpu_launches"] = args.steps * (1 + 1 + 5 + 5)
+    res["gpu_launches"] = extra_steps(args) * (1 + 1 + 5 + 5)
     return res
 
 
@@ -423,7 +442,7 @@ def run_sparse(args, dev, flush, pk):
     for _ in range(args.warmup):
         flush.zero_()
         dec.decode(q, pool, bt, sl, ix, wl.softmax_scale, out, lse)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(extra_steps(args))]
     torch.cuda.synchronize()
     for a, b in evs:
         flush.zero_()
@@ -457,7 +476,7 @@ def run_sparse(args, dev, flush, pk):
                          "frac": gbs / pk["hbm_gbs"], "bytes": nbytes,
                          "note": "bytes of a fused design (each listed row read once); this composition moves "
                                  "each row three times"},
-            "gpu_launches": 4 * args.steps, "cpu_baseline": cpu}
+            "gpu_launches": 4 * extra_steps(args), "cpu_baseline": cpu}
 
 
 def var6_flops(b, h, s, t, n):
@@ -488,7 +507,7 @@ def run_var6(args, dev, flush, pk):
         for _ in range(args.warmup):
             flush.zero_()
             fn()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(extra_steps(args))]
         torch.cuda.synchronize()
         for a, e in evs:
             flush.zero_()
@@ -520,7 +539,7 @@ def run_var6(args, dev, flush, pk):
                              "tflops": var6_flops(b, h, s, t, n) / (us * 1e-6) / 1e12})
     if dec.status() != 0:
         raise RuntimeError("device status set in the latent-path timing")
-    res["gpu_launches"] = args.steps * (4 + 2 * 6)
+    res["gpu_launches"] = extra_steps(args) * (4 + 2 * 6)
     return res
 
 
@@ -547,74 +566,183 @@ def run_projections_only(args, wl, world, rank):
         print(json.dumps(res), flush=True)
 
 
-def run_ours(args, wl, world, rank, local):
-    import mla_latent_space_b200 as mla
-    from mla_latent_space_b200 import build
-    build.build()
-    dev = torch.device("cuda", torch.cuda.current_device())
-    shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages, wl.cache_dtype, wl.causal)
-    q = wl.q.to(dev)
-    pool = wl.pool.to(dev)
-    kv_scale = None if wl.kv_scale is None else wl.kv_scale.to(dev)
-    bt = torch.from_numpy(wl.block_table).to(dev)
-    sl = torch.from_numpy(wl.seqlens).to(dev)
-    out = torch.empty((wl.batch, wl.s_q, wl.num_heads, 512), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((wl.batch, wl.s_q, wl.num_heads), dtype=torch.float32, device=dev)
-    dec = mla.Decoder(shape, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    decode_fn = mla.mla_decode_fwd_simt if args.simt else mla.mla_decode_fwd
-    stream = torch.cuda.current_stream()
+class DeviceWorkload:
+    """One workload's inputs and outputs resident on the GPU, with its
+    decoder (schedule and workspace)."""
 
-    def step(ev=None):
-        dec.schedule(sl)
+    def __init__(self, wl, dev):
+        import mla_latent_space_b200 as mla
+        self.wl = wl
+        self.shape = mla.make_shape(wl.batch, wl.s_q, wl.num_heads, wl.max_pages, wl.num_pages, wl.cache_dtype,
+                                    wl.causal)
+        self.q = wl.q.to(dev)
+        self.pool = wl.pool.to(dev)
+        self.kv_scale = None if wl.kv_scale is None else wl.kv_scale.to(dev)
+        self.bt = torch.from_numpy(wl.block_table).to(dev)
+        self.sl = torch.from_numpy(wl.seqlens).to(dev)
+        self.out = torch.empty((wl.batch, wl.s_q, wl.num_heads, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((wl.batch, wl.s_q, wl.num_heads), dtype=torch.float32, device=dev)
+        self.dec = mla.Decoder(self.shape, device=dev)
+
+    def step(self, ev=None):
+        """schedule -> decode -> combine; `ev` brackets the decode launch."""
+        import mla_latent_space_b200 as mla
+        stream = torch.cuda.current_stream()
+        d, wl = self.dec, self.wl
+        d.schedule(self.sl)
         if ev is not None:
             ev[0].record(stream)
-        decode_fn(shape, q, pool, kv_scale, bt, sl, wl.softmax_scale, dec.sched, dec.workspace, out, lse)
+        mla.mla_decode_fwd(self.shape, self.q, self.pool, self.kv_scale, self.bt, self.sl, wl.softmax_scale,
+                           d.sched, d.workspace, self.out, self.lse)
         if ev is not None:
             ev[1].record(stream)
-        mla.mla_combine(shape, dec.sched, dec.workspace, out, lse)
+        mla.mla_combine(self.shape, d.sched, d.workspace, self.out, self.lse)
 
-    for _ in range(args.warmup):
+    def status(self):
+        return self.dec.status()
+
+
+def time_steps(args, dw, flush, K, world=1, local=0, sample_clocks=False):
+    """W warm-up steps, then K timed steps (L2 flushed before each, outside
+    the events), then K more with events around the decode launch alone.
+    Returns (step ms list, decode ms list, clocks or None)."""
+    import mla_latent_space_b200 as mla
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
         flush.zero_()
-        step()
+        dw.step()
     torch.cuda.synchronize()
-    st = dec.status()
+    st = dw.status()
     if st != 0:
-        raise RuntimeError(f"device status after warm-up: {mla.error_string(st)}")
-
-    K = args.steps
+        raise RuntimeError(f"{dw.wl.name}: device status after warm-up: {mla.error_string(st)}")
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
+    clocks = ClockSampler(local) if sample_clocks else None
     barrier(world)
     torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
     # the step is bracketed by events only at its ends: an event between two
     # of its kernels would stop the next one from launching behind the
     # previous (programmatic dependent launch)
     for k in range(K):
-        flush.zero_()                       # L2 flush outside the timed events
+        flush.zero_()
         ev_step[k][0].record(stream)
-        step()
+        dw.step()
         ev_step[k][1].record(stream)
     torch.cuda.synchronize()
     # the decode kernel alone, for the roofline: the same steps with events
     # around the decode launch
     for k in range(K):
         flush.zero_()
-        step(ev_dec[k])
+        dw.step(ev_dec[k])
     torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
     barrier(world)
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev_step]
-    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    st = dw.status()
+    if st != 0:
+        raise RuntimeError(f"{dw.wl.name}: device status after timing: {mla.error_string(st)}")
+    return [a.elapsed_time(b) for a, b in ev_step], [a.elapsed_time(b) for a, b in ev_dec], clk
+
+
+def roofline(wl, dec_ms, pk, pk_kind, traffic):
+    """The decode kernel against the bound the cost model picks for this
+    workload: HBM when its bytes take longer at the measured copy bandwidth
+    than its FLOPs at the measured bf16 GEMM rate, else the tensor core."""
+    flops, nbytes = cost.workload_cost(wl)
+    gbs = nbytes / (dec_ms * 1e-3) / 1e9
+    tflops = flops / (dec_ms * 1e-3) / 1e12
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                "traffic": traffic}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tflops / pk["bf16_tflops"], "traffic": traffic}
+    roof["kernel"] = "mla_decode_fwd"
+    roof["peak_kind"] = f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback"
+    roof["launch_us"] = dec_ms * 1e3
+    roof["roofline_us"] = max(t_hbm, t_tc) * 1e6
+    roof["tensor_frac"] = tflops / pk["bf16_tflops"]
+    roof["tensor_frac_sustained"] = tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    roof["hbm_frac"] = gbs / pk["hbm_gbs"]
+    if wl.cache_dtype == "fp8":
+        roof["note"] = ("the cost model's bf16 tensor peak, as for the other workloads; the latent scores run "
+                        "as FP8 MMAs, the value product as fp16 MMAs")
+    return roof
+
+
+def oracle_timed(wl, budget_s):
+    """The fp64 oracle over whole requests (every query token, every head)
+    in batch order until `budget_s` seconds have passed (at least one
+    request).  Returns (TFLOP/s, seconds, description)."""
+    import oracle
+    t_tot, fl, n = 0.0, 0.0, 0
+    while n < wl.batch and (n == 0 or t_tot < budget_s):
+        rows = [(n, i) for i in range(wl.s_q)]
+        t0 = time.perf_counter()
+        oracle.decode(wl, rows=rows)
+        t_tot += time.perf_counter() - t0
+        fl += cost.mla_flops(1, wl.num_heads, wl.s_q, None, sum_t=int(wl.seqlens[n]))
+        n += 1
+    toks = int(wl.seqlens[:n].astype(np.int64).sum())
+    return fl / t_tot / 1e12, t_tot, f"requests 0..{n - 1} of {wl.batch} ({toks} cached tokens, all heads)"
+
+
+def per_config(args, dev, flush, pk, pk_kind, headline=None):
+    """The five workloads, each timed like the headline (schedule -> decode
+    -> combine with the L2 flushed before every step) with its decode launch
+    against its roofline, and the oracle on a bounded sample of it."""
+    res = {}
+    K = max(5, min(args.steps, args.per_config_steps))
+    for cfg in (1, 2, 3, 4, 5):
+        if headline is not None and cfg == args.config:
+            wl, step_ms, dec_ms = headline
+        else:
+            wl = mw.make_config(cfg, seed=0)
+            dw = DeviceWorkload(wl, dev)
+            step_ms, dec_ms, _ = time_steps(args, dw, flush, K)
+            del dw
+            torch.cuda.empty_cache()
+        flops, nbytes = cost.workload_cost(wl)
+        us = sum(step_ms) / len(step_ms) * 1e3
+        dus = sum(dec_ms) / len(dec_ms) * 1e3
+        ent = {"workload": wl.name, "steps": len(step_ms), "us_per_step": us,
+               "tflops": flops / (us * 1e-6) / 1e12, "kv_gbs": nbytes / (us * 1e-6) / 1e9,
+               "decode_us": dus, "flops": flops, "bytes": nbytes,
+               "roofline": roofline(wl, dus * 1e-3, pk, pk_kind, captured_traffic(wl.name))}
+        if cfg == 1:
+            ent["note"] = "0.66 MB and 18 MFLOP: launch-bound, reported only"
+        if not args.no_cpu_baseline:
+            tf, sec, desc = oracle_timed(wl, args.cpu_seconds)
+            ent["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                   "sample": desc, "seconds": sec}
+        res[f"config{cfg}"] = ent
+        del wl
+    return res, 3 * 2 * K * 4   # launches of the timed regions of the four re-timed workloads
+
+
+def config_dict(wl, world):
+    """The `config` of the JSON line; both arms print the same one."""
+    return {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.num_heads,
+            "seq_len": int(wl.seqlens.max()), "sum_t": wl.total_tokens, "page": 64, "cache": wl.cache_dtype,
+            "causal": bool(wl.causal), "parallelism": f"replicas x{world}",
+            "l2": "flushed before every timed step (256 MiB write, outside the events)"}
+
+
+def run_ours(args, wl, world, rank, local):
+    import mla_latent_space_b200 as mla
+    from mla_latent_space_b200 import build
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dw = DeviceWorkload(wl, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K = args.steps
+    step_ms, dec_ms, clk = time_steps(args, dw, flush, K, world=world, local=local, sample_clocks=True)
     my_ms = sum(step_ms) / K
     ms = max_over_ranks(my_ms, world)
     dec_avg_ms = sum(dec_ms) / K
-    st = dec.status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {mla.error_string(st)}")
 
     # End to end through the public API with host buffers.  Every step copies
     # its query, block table and lengths host -> device (pinned memory) and
@@ -624,55 +752,40 @@ def run_ours(args, wl, world, rank, local):
     # overlap step k+1's upload and step k-1's download (a step's kernels
     # wait for its upload; a buffer is reused only after the step that last
     # used it has been downloaded).  The cache (302 MB) is larger than L2.
-    e2e_ms = run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world)
-    # the extras (the rows around the decode) are timed in single-GPU runs; a
-    # multi-GPU run measures the headline step on every replica
+    e2e_ms = run_e2e_pipelined(args, wl, dev, dw.shape, dw.pool, dw.kv_scale, world)
+    # the extras (the other workloads and the rows around the decode) are
+    # timed in single-GPU runs; a multi-GPU run measures the headline step on
+    # every replica
     extras = world == 1
-    proj = run_projections(args, wl, dev, shape, pool, kv_scale, bt, sl, flush, peaks()[0]) \
+    pk, pk_kind = peaks()
+    proj = run_projections(args, wl, dev, dw.shape, dw.pool, dw.kv_scale, dw.bt, dw.sl, flush, pk) \
         if extras and not args.no_projections else None
-    sparse = run_sparse(args, dev, flush, peaks()[0]) if extras and not args.no_sparse else None
-    var6 = run_var6(args, dev, flush, peaks()[0]) if extras and not args.no_var6 else None
+    sparse = run_sparse(args, dev, flush, pk) if extras and not args.no_sparse else None
+    var6 = run_var6(args, dev, flush, pk) if extras and not args.no_var6 else None
     h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
+    del dw
+    torch.cuda.empty_cache()
+    pcfg, pc_launches = per_config(args, dev, flush, pk, pk_kind, headline=(wl, step_ms, dec_ms)) \
+        if extras and not args.no_per_config else (None, 0)
 
     flops, nbytes = cost.workload_cost(wl)
-    pk, pk_kind = peaks()
     value = world * flops / (ms * 1e-3) / 1e12
-    dec_gbs = nbytes / (dec_avg_ms * 1e-3) / 1e9
-    dec_tflops = flops / (dec_avg_ms * 1e-3) / 1e12
-    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
-    t_tc = flops / (pk["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
-    traffic = args.traffic
-    if traffic is None and not args.simt:
-        traffic = captured_traffic(wl.name)
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": dec_gbs / pk["hbm_gbs"], "traffic": traffic}
-    else:
-        roof = {"bound": "tensor", "achieved": dec_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": dec_tflops / pk["bf16_tflops"], "traffic": traffic}
-    roof["kernel"] = "mla_decode_fwd (simt debug path)" if args.simt else "mla_decode_fwd"
-    roof["peak_kind"] = f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback"
-    roof["launch_us"] = dec_avg_ms * 1e3
-    roof["tensor_frac"] = dec_tflops / pk["bf16_tflops"]
-    roof["tensor_frac_sustained"] = dec_tflops / pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-
+    traffic = args.traffic if args.traffic is not None else captured_traffic(wl.name)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.batch, "s_q": wl.s_q, "heads": wl.num_heads,
-                       "seq_len": int(wl.seqlens.max()), "sum_t": wl.total_tokens, "page": 64,
-                       "cache": wl.cache_dtype, "parallelism": f"replicas x{world}",
-                       "l2": "flushed before every timed step (256 MiB write, outside the events)"},
+            "config": config_dict(wl, world),
             "kv_gbs": world * nbytes / (ms * 1e-3) / 1e9,
             "us_per_step": ms * 1e3,
-            "roofline": roof,
+            "roofline": roofline(wl, dec_avg_ms, pk, pk_kind, traffic),
             "clocks": clk,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers"},
             "gpu_launches": 3 * K}
+    if pcfg is not None:
+        line["per_config"] = pcfg
     if proj is not None:
         line["mla_attention"] = proj
     if sparse is not None:
@@ -680,14 +793,13 @@ def run_ours(args, wl, world, rank, local):
     if var6 is not None:
         line["mlavar6"] = var6
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # about 10 s of oracle work: the sample repeated until 10 s have passed
-        n_req = max(1, min(wl.batch, args.ref_requests))
-        tot_dt, tot_fl, reps = 0.0, 0.0, 0
-        while tot_dt < 10.0 and reps < 50:
-            dt, fl, desc = oracle_sample(wl, n_req)
-            tot_dt, tot_fl, reps = tot_dt + dt, tot_fl + fl, reps + 1
-        line["cpu_baseline"] = {"value": tot_fl / tot_dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-                                "kind": "oracle", "sample": f"{desc}, x{reps}", "seconds": tot_dt}
+        if pcfg is not None:
+            cb = dict(pcfg[f"config{args.config}"]["cpu_baseline"])
+        else:
+            tf, sec, desc = oracle_timed(wl, args.cpu_seconds)
+            cb = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle", "sample": desc,
+                  "seconds": sec}
+        line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -695,11 +807,14 @@ def run_ours(args, wl, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2, help="workload 1-5 (2 = the headline decode batch)")
-    ap.add_argument("--simt", action="store_true", help="time the SIMT debug kernel instead")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the five-workload block")
+    ap.add_argument("--per-config-steps", type=int, default=50, help="timed steps of each per-config workload")
+    ap.add_argument("--cpu-seconds", type=float, default=3.0, help="oracle seconds per cpu_baseline sample")
+    ap.add_argument("--ref-seconds", type=float, default=5.0, help="oracle seconds per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-projections", action="store_true",
                     help="skip the timing of the query absorption / output decompression kernels")
@@ -709,7 +824,6 @@ def main():
     ap.add_argument("--sparse-only", action="store_true", help="time only the token-level sparse decode")
     ap.add_argument("--no-var6", action="store_true", help="skip the timing of the MLAvar6+ split decode")
     ap.add_argument("--e2e-buffers", type=int, default=3, help="buffer sets of the pipelined end-to-end loop")
-    ap.add_argument("--ref-requests", type=int, default=64, help="requests in the oracle's timed sample")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per decode launch for the current kernel (else null)")
     args = ap.parse_args()

@@ -49,7 +49,8 @@ enum {
   MLA_ERR_WORKSPACE = -3,    /* workspace / schedule buffer too small          */
   MLA_ERR_CUDA = -4,         /* a CUDA runtime call failed (launch, attribute) */
   MLA_ERR_TIMEOUT = -5,      /* device status: a bounded wait gave up          */
-  MLA_ERR_DEVICE_CHECK = -6  /* device status: seqlen / page id out of range   */
+  MLA_ERR_DEVICE_CHECK = -6  /* device status: seqlen / page id out of range,
+                                or a value row outside fp16's range            */
 };
 
 /* ---- cache element types -------------------------------------------------- */
@@ -121,6 +122,10 @@ int mla_get_schedule(const mla_shape_t* shape, const int32_t* seqlens, int num_s
  *                page holding tokens 64j..64j+63 of request r.  Entries past
  *                ceil(visible/64) are never read.  Out-of-range page ids are
  *                skipped and flagged (MLA_ERR_DEVICE_CHECK).
+ *                The PV product runs in fp16: a value entry (or, FP8, an
+ *                e4m3 value times its scale) of magnitude 65520 or more, or
+ *                a NaN / infinity, is flagged (MLA_ERR_DEVICE_CHECK) and the
+ *                output of the tiles that read it is not valid.
  *   seqlens    : the same int32 [batch] array given to mla_get_schedule.
  *   softmax_scale : multiplies the raw 576-d dot product before softmax.
  *   sched      : filled by mla_get_schedule for this shape and num_sms.
@@ -151,18 +156,10 @@ int mla_decode_fwd(const mla_shape_t* shape, const void* q, const void* kv_cache
 int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace,
                 size_t workspace_bytes, void* out, float* lse, void* stream);
 
-/* Debug path, used by the tests only: the same decode computed by a plain
- * SIMT kernel (fp32 FMA, no tensor cores) over the same schedule and
- * workspace.  Never chosen by mla_decode_fwd. */
-int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_cache,
-                        const float* kv_scale, const int32_t* block_table,
-                        const int32_t* seqlens, float softmax_scale, const void* sched,
-                        void* workspace, size_t workspace_bytes, void* out, float* lse,
-                        void* stream);
-
 /* Reads and clears the sticky device status words that the scheduler and
  * the decode kernels set instead of trapping (a bounded wait that gave up,
- * an out-of-range seqlen or page id).  SYNCHRONISES `stream`.  *status
+ * an out-of-range seqlen or page id, a value row outside fp16's range).
+ * SYNCHRONISES `stream`.  *status
  * receives MLA_OK, MLA_ERR_TIMEOUT or MLA_ERR_DEVICE_CHECK. */
 int mla_get_device_status(const void* sched, void* workspace, void* stream, int* status);
 
@@ -190,6 +187,13 @@ int mla_plan_schedule_host(const mla_shape_t* shape, const int32_t* seqlens, int
  *   (4-byte aligned) that receives, in stream order, this call's status
  *   word (0, or the bits behind MLA_ERR_TIMEOUT / MLA_ERR_DEVICE_CHECK);
  *   NULL to skip.  The call zeroes the status word before its kernels run.
+ * Every check that can fail on the host (arguments, the tile limit, the
+ * tensor-map encoding) is made before the first enqueue, so those errors
+ * leave nothing on the stream; only a failing kernel launch itself
+ * (MLA_ERR_CUDA) can leave this call's earlier kernels enqueued.
+ * The static array's address is cached per device for the life of the
+ * process; calling this after cudaDeviceReset on a device it was used on is
+ * not supported.
  * Calls that overlap in time on one device (different streams, or threads
  * without ordering) share the static array and race: serialise them. */
 int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, const void* kv_cache,

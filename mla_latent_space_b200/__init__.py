@@ -26,7 +26,7 @@ D_HEAD, D_ROPE = 128, 64   # per-head dims before absorption, RoPE dims
 FP8_PAGE_BYTES = PAGE * D_V + PAGE * (D_QK - D_V) * 2
 
 EXPORTED = ("mla_schedule_bytes", "mla_workspace_bytes", "mla_get_schedule", "mla_decode_fwd",
-            "mla_combine", "mla_decode_fwd_simt", "mla_get_device_status", "mla_plan_schedule_host",
+            "mla_combine", "mla_get_device_status", "mla_plan_schedule_host",
             "mla_error_string", "mla_version", "mla_decode_fwd_noalloc")
 
 
@@ -62,8 +62,6 @@ def lib() -> ctypes.CDLL:
         dec = [sp, vp, vp, vp, vp, vp, f32, vp, vp, sz, vp, vp, vp]
         L.mla_decode_fwd.argtypes = dec
         L.mla_decode_fwd.restype = i32
-        L.mla_decode_fwd_simt.argtypes = dec
-        L.mla_decode_fwd_simt.restype = i32
         L.mla_combine.argtypes = [sp, vp, vp, sz, vp, vp, vp]
         L.mla_combine.restype = i32
         L.mla_get_device_status.argtypes = [vp, vp, vp, ctypes.POINTER(i32)]
@@ -208,12 +206,6 @@ def mla_decode_fwd(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_s
                    stream=None):
     _decode_common(lib().mla_decode_fwd, "mla_decode_fwd", shape, q, kv_cache, kv_scale, block_table, seqlens,
                    softmax_scale, sched, workspace, out, lse, stream)
-
-
-def mla_decode_fwd_simt(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace, out,
-                        lse, stream=None):
-    _decode_common(lib().mla_decode_fwd_simt, "mla_decode_fwd_simt", shape, q, kv_cache, kv_scale, block_table,
-                   seqlens, softmax_scale, sched, workspace, out, lse, stream)
 
 
 def mla_decode_fwd_noalloc(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, out, lse,
@@ -371,8 +363,10 @@ class Decoder:
         mla_get_schedule(self.shape, seqlens, self.n_sms, self.sched, stream)
 
     def decode(self, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, out, lse, stream=None,
-               simt=False):
-        fn = mla_decode_fwd_simt if simt else mla_decode_fwd
+               decode_fn=None):
+        """Decode + combine.  ``decode_fn`` replaces mla_decode_fwd (same
+        signature); the tests pass the SIMT kernel of the test library."""
+        fn = mla_decode_fwd if decode_fn is None else decode_fn
         fn(self.shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, self.sched, self.workspace,
            out, lse, stream)
         mla_combine(self.shape, self.sched, self.workspace, out, lse, stream)

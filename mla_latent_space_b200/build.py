@@ -5,6 +5,11 @@
 The library statically links the CUDA runtime, so at run time it needs only
 the driver.  Rebuilds when any source under csrc/ or include/ is newer than
 the library.
+
+A second library, libmla_b200_test.so, is built beside it for the tests
+only: the same objects plus the SIMT decode kernel, with the C-ABI file
+compiled under MLA_TEST_ENTRY_POINTS so that it also exports
+mla_decode_fwd_simt.  The product library does not contain that kernel.
 """
 from __future__ import annotations
 
@@ -17,6 +22,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmla_b200.so")
+TEST_LIB = os.path.join(HERE, "libmla_b200_test.so")
+TEST_ONLY = ("decode_simt.cu",)        # compiled into the test library alone
+TEST_FLAGGED = ("api.cu",)             # compiled a second time with MLA_TEST_ENTRY_POINTS
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -26,14 +34,14 @@ def sources():
 
 
 def _deps():
-    return (sources() + glob.glob(os.path.join(CSRC, "*.cuh"))
+    return (sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
             + glob.glob(os.path.join(ROOT, "include", "*.h")) + [os.path.abspath(__file__)])
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(TEST_LIB)):
         return False
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(TEST_LIB))
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -44,15 +52,18 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     os.makedirs(objdir, exist_ok=True)
     flags = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
                     "-I" + os.path.join(ROOT, "include"), *extra]
-    objs = []
-    procs = []
+    jobs = []   # (source, object, extra flags)
     for src in sources():
-        obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *flags, "-c", src, "-o", obj]
+        base = os.path.basename(src)
+        jobs.append((src, os.path.join(objdir, base + ".o"), []))
+        if base in TEST_FLAGGED:
+            jobs.append((src, os.path.join(objdir, base + ".test.o"), ["-DMLA_TEST_ENTRY_POINTS"]))
+    procs = []
+    for src, obj, fl in jobs:
+        cmd = [NVCC, *flags, *fl, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
-        objs.append(obj)
     failed = []
     for src, p in procs:
         out = p.communicate()[0].decode()
@@ -63,10 +74,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if failed:
         msg = "\n".join(f"--- {s}\n{o}" for s, o in failed)
         raise RuntimeError("nvcc failed:\n" + msg)
-    tmp = LIB + ".tmp"
-    cmd = [NVCC, *ARCH, "-shared", "--cudart", "static", "-o", tmp, *objs, "-lrt", "-ldl", "-lpthread"]
-    subprocess.run(cmd, check=True, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
-    os.replace(tmp, LIB)
+    product = [o for s_, o, fl in jobs if not fl and os.path.basename(s_) not in TEST_ONLY]
+    test = [o for s_, o, fl in jobs if fl or os.path.basename(s_) not in TEST_FLAGGED]
+    for lib, objs in ((LIB, product), (TEST_LIB, test)):
+        tmp = lib + ".tmp"
+        cmd = [NVCC, *ARCH, "-shared", "--cudart", "static", "-o", tmp, *objs, "-lrt", "-ldl", "-lpthread"]
+        subprocess.run(cmd, check=True, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
+        os.replace(tmp, lib)
     return LIB
 
 

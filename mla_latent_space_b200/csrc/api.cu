@@ -7,20 +7,22 @@
 #include <cstring>
 #include <mutex>
 
-#include "common.cuh"
+#include "decode_launch.cuh"
+#ifdef MLA_TEST_ENTRY_POINTS
+#include "test_entry.h"
+#endif
 
 namespace mla {
 void plan_schedule_host(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched);
 cudaError_t launch_schedule(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched, cudaStream_t st);
+#ifdef MLA_TEST_ENTRY_POINTS
 cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_scale, const int32_t* block_table,
                                const int32_t* seqlens, float scale, const void* sched, void* ws, void* out,
                                float* lse, int num_pages, int fp8, int cap_slots, int grid_ctas,
                                cudaStream_t stream);
+#endif
 cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
                            int cap_slots, cudaStream_t stream);
-int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
-                        const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
-                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
 cudaError_t launch_sparse_gather(const int32_t* indices, int topk, const int32_t* seqlens, int batch, int s_q,
                                  const int32_t* block_table, int max_pages, int num_pages, const void* pool,
                                  const float* kv_scale, void* scratch, float* vscale, int vpages, int32_t* vseqlens,
@@ -245,6 +247,9 @@ int mla_decode_fwd(const mla_shape_t* shape, const void* q, const void* kv_cache
                              cap_slots_for(workspace_bytes), out, lse, static_cast<cudaStream_t>(stream));
 }
 
+#ifdef MLA_TEST_ENTRY_POINTS
+// Test-only entry point (built into the test library alone): the SIMT
+// decode kernel over the same schedule and workspace.
 int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_cache, const float* kv_scale,
                         const int32_t* block_table, const int32_t* seqlens, float softmax_scale,
                         const void* sched, void* workspace, size_t workspace_bytes, void* out, float* lse,
@@ -259,6 +264,7 @@ int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_
                                      cap_slots_for(workspace_bytes), sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
+#endif
 
 int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace, size_t workspace_bytes,
                 void* out, float* lse, void* stream) {
@@ -441,7 +447,7 @@ const char* mla_error_string(int code) {
     case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: schedule or workspace buffer too small";
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
     case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device wait gave up";
-    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: out-of-range seqlen or page id seen on the device";
+    case MLA_ERR_DEVICE_CHECK: return "MLA_ERR_DEVICE_CHECK: out-of-range seqlen or page id, or a value row outside fp16 range, seen on the device";
     default: return "MLA: unknown error code";
   }
 }

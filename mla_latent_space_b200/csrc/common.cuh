@@ -42,7 +42,7 @@ constexpr int32_t kStatusTimeout = 1;
 constexpr int32_t kStatusBadSeqlen = 2;
 constexpr int32_t kStatusBadPage = 4;
 constexpr int32_t kStatusWorkspace = 8;
-constexpr int32_t kStatusBadInput = 16;   // reserved (set by no kernel at present)
+constexpr int32_t kStatusBadInput = 16;   // a cache value the decode cannot represent (V outside fp16)
 
 // ---------------------------------------------------------------------------
 // workspace: [256 B status][max_slots x 128 x 512 fp32 O][max_slots x 128 fp32 lse]

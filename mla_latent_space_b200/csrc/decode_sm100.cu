@@ -52,6 +52,7 @@
 
 #include <mutex>
 
+#include "decode_launch.cuh"
 #include "kernel_util.cuh"
 #include "sm100_ptx.cuh"
 
@@ -181,48 +182,8 @@ struct Params {
   int num_pages;
   int cap_slots;
   int q_rows;         // batch * s_q * heads
-  unsigned long long* trace;   // event trace (builds with MLA_TRACE only)
 };
 
-// Optional device event trace.  Built only with -DMLA_TRACE: one thread per
-// role of cluster 0 records (event << 24 | index, clock64, 0) into
-// trace[role][2048][3]; the last entry of roles 6 and 7 holds one
-// (0, clock64, %globaltimer) pair per CTA taken right after the start-up
-// cluster barrier, to line the two SMs' clocks up.  Only the SM clock is
-// read per event (the global timer
-// is far slower to read and would distort the timeline).  In normal builds
-// the hooks compile to nothing.
-#ifdef MLA_TRACE
-#ifndef MLA_TRACE_CLUSTER
-#define MLA_TRACE_CLUSTER 0
-#endif
-#define MLA_TR(role, ev, j)                                                               \
-  do {                                                                                    \
-    if (p.trace && cluster_id_x() == MLA_TRACE_CLUSTER) {                                                 \
-      const unsigned k_ = trk_++;                                                         \
-      if (k_ < 2047) {                                                                    \
-        unsigned long long* e_ = p.trace + (size_t(role) * 2048 + k_) * 3;                \
-        e_[0] = (unsigned long long)(((ev) << 24) | (unsigned(j) & 0xFFFFFF));            \
-        e_[1] = clock64();                                                                \
-      }                                                                                   \
-    }                                                                                     \
-  } while (0)
-#define MLA_TR_SYNC(role)                                                                 \
-  do {                                                                                    \
-    if (p.trace && cluster_id_x() == MLA_TRACE_CLUSTER) {                                                 \
-      unsigned long long* e_ = p.trace + (size_t(role) * 2048 + 2047) * 3;                \
-      e_[1] = clock64();                                                                  \
-      e_[2] = globaltimer();                                                              \
-    }                                                                                     \
-  } while (0)
-#else
-#define MLA_TR(role, ev, j) \
-  do {                      \
-  } while (0)
-#define MLA_TR_SYNC(role) \
-  do {                    \
-  } while (0)
-#endif
 
 struct Ctl {
   volatile int32_t* abort;
@@ -335,8 +296,19 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled(uint32_t two, __half2 scale) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// bf16 pair -> fp16 pair (exact inside fp16's range); *big records a value
-// outside it (or NaN).
+// Running max of |h| over fp16 pairs, NaN-propagating: a converted V value
+// that left fp16's finite range (a bf16 value of magnitude 65520 or more, an
+// infinite or NaN input, an FP8 value times a scale above the range) leaves
+// an infinity or a NaN here.
+__device__ __forceinline__ void track_absmax(__half2& acc, uint32_t w) {
+  acc = __hmax2_nan(acc, __habs2(*reinterpret_cast<const __half2*>(&w)));
+}
+
+__device__ __forceinline__ bool absmax_finite(__half2 acc) {
+  const float2 f = __half22float2(acc);
+  return f.x <= 65504.f && f.y <= 65504.f;   // false for inf and NaN
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc], kind::f8f6f4 (the FP8 cache's latent scores).
 __device__ __forceinline__ void mma_ts_f8(uint32_t d, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -426,16 +398,17 @@ __device__ __forceinline__ int conv_rank(int warp) {
 }
 
 // Calls f(piece) for every piece of every worker this cluster owns; stops
-// when f returns false.
+// when f returns false.  Returns true when every call returned true.
 template <class F>
-__device__ __forceinline__ void each_piece(const SchedView& sv, F&& f) {
+__device__ __forceinline__ bool each_piece(const SchedView& sv, F&& f) {
   const int ncl = int(nclusters_x());
   for (int w = int(cluster_id_x()); w < sv.W; w += ncl) {
     PieceIter it(sv, w);
     Piece pc;
     while (it.next(&pc))
-      if (!f(pc)) return;
+      if (!f(pc)) return false;
   }
+  return true;
 }
 
 __device__ __forceinline__ int clamp_len(int t, const SchedView& sv) {
@@ -458,7 +431,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-  [[maybe_unused]] unsigned trk_ = 0;   // trace builds: this thread's event count (one recording thread per role)
 
   if (tid == 0) {
     // FP8 cache: a ring stage is refilled once the softmax and the issuer
@@ -516,7 +488,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
   const int rows_total = sv.s_q * sv.heads;
 
   Ctl ctl{&bars->abort, mapa(smem_u32(&bars->abort), rank ^ 1u), p.ws};
-  if (tid == 0) MLA_TR_SYNC(6 + rank);
 
   if (rank == 0) {
     // ======================= score CTA =======================
@@ -541,7 +512,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const uint32_t s = zc % nz, ph = (zc / nz) & 1u;
           if (!ewait(ctl, bar(bars->z_empty[s]), ph ^ 1u)) return false;
           if (leader) {
-            MLA_TR(0, 1, zc);
             mbar_arrive_expect_tx(bar(bars->z_full[s]), tx);
           }
           *dst = sbase + L::z + s * L::zbytes;
@@ -674,7 +644,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         }
         if (!ewait(ctl, bar(bars->q_ready), pieces & 1u)) return false;
         if (kFp8 && !ewait(ctl, bar(bars->qpe_full), pieces & 1u)) return false;
-        if (leader) MLA_TR(1, 0, bc);
         ++pieces;
         // the query rows are in TMEM: release their stages
         if constexpr (!kFp8) {
@@ -685,13 +654,11 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         tc_fence_after();
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
           if (!ewait(ctl, bar(bars->s_empty), (bc & 1u) ^ 1u)) return false;
-          if (leader) MLA_TR(1, 2, bc);
           tc_fence_after();
           if constexpr (kFp8) {
             {
               const uint32_t zs = zc % nz;
               if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-              if (leader) MLA_TR(1, 20, zc);
               tc_fence_after();
               const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
               const uint32_t d = tmem + kTmemS;
@@ -711,7 +678,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             for (int e = 0; e < 4; ++e, ++zc) {
               const uint32_t zs = zc % nz;
               if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-              if (leader) MLA_TR(1, 21, zc);
               tc_fence_after();
               const uint64_t bd = zdesc0 + uint64_t(zs * (kZStage >> 4));
               const uint32_t d = tmem + kTmemSLat;
@@ -730,7 +696,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             for (int q = 0; q < 5; ++q, ++zc) {
               const uint32_t zs = zc % nz;
               if (!ewait(ctl, bar(bars->z_full[zs]), (zc / nz) & 1u)) return false;
-              if (leader) MLA_TR(1, 10 + q, bc);
               tc_fence_after();
               const uint32_t d = tmem + kTmemS;
               if (leader) {
@@ -753,7 +718,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           if (leader) {
             mma_commit(bar(bars->s_full));
-            MLA_TR(1, 3, bc);
           }
           __syncwarp();
         }
@@ -782,7 +746,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
         const bool valid = rho < rows_total;
         const int t = clamp_len(p.seqlens[r], sv);
         const int Lrow = valid ? visible_len(t, sv.s_q, rho / sv.heads, sv.causal) : 0;
-        if (g == 0) MLA_TR(2, 9, bc);
         // query row i -> TMEM lane i.  Box c of the query (rows 0-63, then
         // 64-127 at +8 KB) is sub-stage c % qbs of stage zc + c / qbs.  BF16
         // cache: boxes 0-8, two per stage, as bf16 pairs in columns [0, 288),
@@ -859,7 +822,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(bars->q_ready));
-          if (g == 0) MLA_TR(2, 0, bc);
         }
         float m = -INFINITY, l = 0.f;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
@@ -875,7 +837,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             if (i < 64) st_shared_u32(scl + 4u * uint32_t(i), __float_as_uint(page >= 0 ? p.kv_scale[size_t(page) * 64 + i] : 0.f));
           }
           if (!gwait(ctl, bar(bars->s_full), bc & 1u, g == 0, carry_ok)) return false;
-          if (g == 0) MLA_TR(2, 1, bc);
           tc_fence_after();
           float x[64];
           {
@@ -930,7 +891,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           // staging is free once the previous block's copy has read it
           if (g == 0) bulk_wait_group_read<0>();
           named_bar_sync(kSoftmaxBar, kSmThreads);
-          if (g == 0) MLA_TR(2, 5, bc);
           const float mb = fmaxf(mh, ld_shared_f32(xmax + 4u * uint32_t(g ^ 128)));
           float m_new = m, alpha = 1.f;
           bool need = false;
@@ -961,7 +921,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                          pack_f16(x[8 * k + 2], x[8 * k + 3]), pack_f16(x[8 * k + 4], x[8 * k + 5]),
                          pack_f16(x[8 * k + 6], x[8 * k + 7]));
           named_bar_sync(kSoftmaxBar, kSmThreads);
-          if (g == 0) MLA_TR(2, 6, bc);
           l = l * alpha + ph + ld_shared_f32(xsum + 4u * uint32_t(g ^ 128));
           m = m_new;
           if (h == 0) {
@@ -977,7 +936,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           const bool two = j + 1 < pc.p1;
           if (g == 0) {
             bool ok = bwait<true>(ctl, bar(bars->x_free[0]), (bc & 1u) ^ 1u);
-            MLA_TR(2, 2, bc);
             if (ok) bulk_copy_to_peer(o_p, stg, kPSlot0, o_pfull);
             if (ok && two) {
               ok = bwait<true>(ctl, bar(bars->x_free[1]), (n1 & 1u) ^ 1u);
@@ -985,7 +943,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             }
             bulk_commit_group();
             carry_ok = ok;
-            MLA_TR(2, 3, bc);
           }
           n1 += two ? 1u : 0u;
         }
@@ -1018,12 +975,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       uint32_t bc = 0, vc = 0, pieces = 0, n1 = 0, nr = 0;
       each_piece(sv, [&](const Piece& pc) {
         if (pieces > 0 && !ewait(ctl, bar(bars->o_free), (pieces - 1) & 1u)) return false;
-        if (leader) MLA_TR(4, 0, bc);
         ++pieces;
         for (int j = pc.p0; j < pc.p1; j += 2, ++bc) {
           const bool two = j + 1 < pc.p1, last = j + 2 >= pc.p1;
           if (!ewait<true>(ctl, bar(bars->p_full[0]), bc & 1u)) return false;
-          if (leader) MLA_TR(4, 1, bc);
           const float4 a4 = ld_shared_f4(meta);
           const float4 l4 = last ? ld_shared_f4(meta + 512u) : make_float4(0.f, 0.f, 0.f, 0.f);
           // re-arm slot 0: its next copy starts only after this block's
@@ -1041,7 +996,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             if (!ewait(ctl, bar(bars->corr_done), nr & 1u)) return false;
             ++nr;
           }
-          if (leader) MLA_TR(4, 2, bc);
           for (int u = 0; u < (two ? 2 : 1); ++u, ++vc) {
             if (u == 1) {
               if (!ewait<true>(ctl, bar(bars->p_full[1]), n1 & 1u)) return false;
@@ -1049,7 +1003,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             }
             const uint32_t vs = vc % NV;
             if (!ewait(ctl, bar(bars->v_full[vs]), (vc / NV) & 1u)) return false;
-            if (leader) MLA_TR(4, 3, vc);
             tc_fence_after();
             const uint64_t ad = pdesc0 + uint64_t((uint32_t(u) * kPSlot0) >> 4);
             const uint64_t bd = vdesc0 + uint64_t((vs * kVStage) >> 4);
@@ -1068,7 +1021,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           n1 += two ? 1u : 0u;
           if (leader) {
             mma_commit(bar(bars->pv_blk[bc % NB]));
-            MLA_TR(4, 4, bc);
           }
           __syncwarp();
           if (last) {
@@ -1105,7 +1057,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           ++ne;
           const uint32_t type = vb->ev_type, eb = vb->ev_blk;
           const float v = vb->ev_val[i];
-          if (i == 0) MLA_TR(5, 1, eb);
           if (type == kEvRescale) {
             // O must hold every earlier block before it is rescaled (never
             // the piece's first block, so eb - 1 exists)
@@ -1131,7 +1082,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           // end of the piece: wait for its last block of PVs, normalise, store
           const uint32_t pb = eb;
           if (!wwait(ctl, bar(bars->pv_blk[pb % NB]), (pb / NB) & 1u)) return false;
-          if (i == 0) MLA_TR(5, 5, eb);
           tc_fence_after();
           const float lfin = v;
           const float inv = lfin > 0.f ? 1.f / lfin : 0.f;
@@ -1168,7 +1118,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
           }
           tc_fence_before();
           mbar_arrive(bar(bars->o_free));
-          if (i == 0) MLA_TR(5, 6, eb);
           return true;
         }
       });
@@ -1209,10 +1158,13 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       // ---- V converters: each landed stage is rewritten in place from bf16
       // to fp16 (same size, same swizzled N-major layout).  Tokens at or
       // past the request's length become zero: their bytes may be anything
-      // and 0 * NaN would poison O.  Thread -> 16 chunks of 16 bytes.
+      // and 0 * NaN would poison O.  Thread -> 16 chunks of 16 bytes.  A
+      // value that does not fit fp16 sets kStatusBadInput (the output of its
+      // tile is then not valid).
       const int ct = conv_rank(warp) * 32 + lane;
       uint32_t vc = 0;
-      each_piece(sv, [&](const Piece& pc) {
+      __half2 vmax = __float2half2_rn(0.f);
+      const bool done = each_piece(sv, [&](const Piece& pc) {
         const int r = pc.T / sv.tiles_per_req;
         const int t = clamp_len(p.seqlens[r], sv);
         for (int j = pc.p0; j < pc.p1; ++j, ++vc) {
@@ -1233,7 +1185,6 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             const float sb = ok ? p.kv_scale[size_t(page) * 64 + ta + 32] : 0.f;
             const bool vwait = ct == 0 ? bwait(ctl, bar(bars->v_loaded[vs]), vph) : true;
             if (!named_bar_and(kConvBar, kConvThreads, vwait)) return false;
-            if (ct == 0) MLA_TR(3, 1, vc);
             uint2 in[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
@@ -1249,33 +1200,43 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
               const uint32_t o = uint32_t(ct + kConvThreads * u), rr = (o & 511u) >> 3;
               if (int(rr) < nvalid) {
                 const __half2 sc = (u & 1) ? hb : ha;
-                st_shared_v4(st + o * 16u, e4m3x2_scaled(in[u].x & 0xFFFFu, sc), e4m3x2_scaled(in[u].x >> 16, sc),
-                             e4m3x2_scaled(in[u].y & 0xFFFFu, sc), e4m3x2_scaled(in[u].y >> 16, sc));
+                const uint32_t a = e4m3x2_scaled(in[u].x & 0xFFFFu, sc), b = e4m3x2_scaled(in[u].x >> 16, sc);
+                const uint32_t c = e4m3x2_scaled(in[u].y & 0xFFFFu, sc), d = e4m3x2_scaled(in[u].y >> 16, sc);
+                track_absmax(vmax, a);
+                track_absmax(vmax, b);
+                track_absmax(vmax, c);
+                track_absmax(vmax, d);
+                st_shared_v4(st + o * 16u, a, b, c, d);
               } else {
                 st_shared_v4(st + o * 16u, 0u, 0u, 0u, 0u);
               }
             }
           } else {
             if (!wwait(ctl, bar(bars->v_loaded[vs]), vph)) return false;
-            if (ct == 0) MLA_TR(3, 1, vc);
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
               const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
               const int tok = int((off & (kBox - 1)) >> 7);
               const uint4 v = ld_shared_v4(st + off);
-              if (tok < nvalid)
-                st_shared_v4(st + off, bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z),
-                             bf16x2_to_f16x2(v.w));
-              else
+              if (tok < nvalid) {
+                const uint32_t a = bf16x2_to_f16x2(v.x), b = bf16x2_to_f16x2(v.y);
+                const uint32_t c = bf16x2_to_f16x2(v.z), d = bf16x2_to_f16x2(v.w);
+                track_absmax(vmax, a);
+                track_absmax(vmax, b);
+                track_absmax(vmax, c);
+                track_absmax(vmax, d);
+                st_shared_v4(st + off, a, b, c, d);
+              } else {
                 st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+              }
             }
           }
           fence_proxy_async_cta();
           mbar_arrive(bar(bars->v_full[vs]));
-          if (ct == 0) MLA_TR(3, 3, vc);
         }
         return true;
       });
+      if (done && !absmax_finite(vmax)) flag_status(p.ws, kStatusBadInput);
     }
   }
 
@@ -1361,37 +1322,31 @@ bool make_q_map(CUtensorMap* map, const void* q, int rows) {
 
 }  // namespace
 
-cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_scale, const int32_t* block_table,
-                               const int32_t* seqlens, float scale, const void* sched, void* ws, void* out,
-                               float* lse, int num_pages, int fp8, int cap_slots, int grid_ctas,
-                               cudaStream_t stream);
 
-int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
-                        const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
-                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream) {
-  int dev = 0, sms = 0;
+int prepare_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, DecodePrepared* pr) {
+  int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MLA_ERR_CUDA;
-  const bool fp8 = shape->cache_dtype == MLA_CACHE_FP8_E4M3;
+  if (cudaDeviceGetAttribute(&pr->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || pr->sms <= 0)
+    return MLA_ERR_CUDA;
+  pr->fp8 = shape->cache_dtype == MLA_CACHE_FP8_E4M3;
   const int q_rows = shape->batch * shape->s_q * shape->num_heads;
-  CUtensorMap pool_map, q_map, rope_map;
-  if (fp8) {
-    if (!make_fp8_maps(&pool_map, &rope_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+  if (pr->fp8) {
+    if (!make_fp8_maps(&pr->pool_map, &pr->rope_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
   } else {
-    if (!make_pool_map(&pool_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
-    rope_map = pool_map;   // not read
+    if (!make_pool_map(&pr->pool_map, kv, shape->num_pages)) return MLA_ERR_CUDA;
+    pr->rope_map = pr->pool_map;   // not read
   }
-  if (!make_q_map(&q_map, q, q_rows)) return MLA_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(decode_sm100_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(kSmemBytes));
-    if (attr_err == cudaSuccess)
-      attr_err = cudaFuncSetAttribute(decode_sm100_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(kSmemBytes));
-  });
-  if (attr_err != cudaSuccess) return MLA_ERR_CUDA;
+  if (!make_q_map(&pr->q_map, q, q_rows)) return MLA_ERR_CUDA;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(pr->fp8 ? &decode_sm100_kernel<true>
+                                                               : &decode_sm100_kernel<false>),
+                        int(kSmemBytes)))
+    return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, const void* q, const void* kv,
+                         const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, float scale,
+                         const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream) {
   Params prm;
   prm.q = static_cast<const uint16_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv);
@@ -1405,9 +1360,8 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.num_pages = shape->num_pages;
   prm.cap_slots = cap_slots;
-  prm.q_rows = q_rows;
-  prm.trace = nullptr;
-  const int clusters = sms / 2 > 0 ? sms / 2 : 1;
+  prm.q_rows = shape->batch * shape->s_q * shape->num_heads;
+  const int clusters = pr.sms / 2 > 0 ? pr.sms / 2 : 1;
   // programmatic dependent launch: the prologue (barriers, TMEM, descriptor
   // prefetch) overlaps the scheduler kernel; the kernel waits for it before
   // reading the schedule
@@ -1421,9 +1375,20 @@ int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = fp8 ? cudaLaunchKernelEx(&cfg, decode_sm100_kernel<true>, pool_map, q_map, rope_map, prm)
-                            : cudaLaunchKernelEx(&cfg, decode_sm100_kernel<false>, pool_map, q_map, rope_map, prm);
+  const cudaError_t e =
+      pr.fp8 ? cudaLaunchKernelEx(&cfg, decode_sm100_kernel<true>, pr.pool_map, pr.q_map, pr.rope_map, prm)
+             : cudaLaunchKernelEx(&cfg, decode_sm100_kernel<false>, pr.pool_map, pr.q_map, pr.rope_map, prm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
+                        const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
+                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream) {
+  DecodePrepared pr;
+  const int rc = prepare_decode_sm100(shape, q, kv, &pr);
+  if (rc != MLA_OK) return rc;
+  return enqueue_decode_sm100(pr, shape, q, kv, kv_scale, block_table, seqlens, scale, sched, ws, cap_slots, out,
+                              lse, stream);
 }
 
 }  // namespace mla

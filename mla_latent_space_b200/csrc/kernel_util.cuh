@@ -7,9 +7,34 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace mla {
+
+// Raises a kernel's dynamic shared-memory limit on the CURRENT device, once
+// per (kernel, device): the attribute is per device, so a process that
+// launches on several GPUs sets it on each of them.  Returns false when the
+// runtime refuses it.  Device ordinals at or above 64 are set on every call.
+inline bool ensure_smem_attr(const void* fn, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  constexpr int kFns = 16;
+  static std::mutex mu;
+  static const void* fns[kFns] = {};
+  static uint64_t done[kFns] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  int i = 0;
+  while (i < kFns && fns[i] != nullptr && fns[i] != fn) ++i;
+  if (i < kFns && fns[i] == fn && dev < 64 && ((done[i] >> dev) & 1u)) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (i < kFns && dev < 64) {
+    fns[i] = fn;
+    done[i] |= uint64_t(1) << dev;
+  }
+  return true;
+}
 
 struct SchedView {
   const int32_t* hdr;

@@ -7,17 +7,15 @@
 
 #include <mutex>
 
-#include "common.cuh"
+#include "decode_launch.cuh"
 
 namespace mla {
 
+size_t schedule_whole_tiles_smem(int num_tiles);
 cudaError_t launch_schedule_whole_tiles(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
                                         int32_t* status, cudaStream_t stream);
 cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
                            int cap_slots, cudaStream_t stream);
-int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
-                        const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
-                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
 
 namespace {
 
@@ -32,7 +30,9 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Address of this device's scratch and its SM count, looked up once per
 // device (the first call on a device, which therefore must not be made while
-// the stream is being captured).
+// the stream is being captured).  The cached address belongs to the device's
+// primary context: after cudaDeviceReset it is stale, and this entry point is
+// not supported in a process that resets a device it has used.
 int scratch_for_device(uint8_t** base, int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MLA_ERR_CUDA;
@@ -102,13 +102,20 @@ extern "C" int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, c
   void* ws = base;
   int32_t* sched = reinterpret_cast<int32_t*>(base + kStatusBytes);
 
+  // every check that can fail on the host comes before the first enqueue, so
+  // an error return leaves nothing of this call on the stream
+  if (schedule_whole_tiles_smem(int(num_tiles)) == 0) return MLA_ERR_WORKSPACE;
+  DecodePrepared prep;
+  rc = prepare_decode_sm100(shape, q, kv_cache, &prep);
+  if (rc != MLA_OK) return rc;
+
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // the status word must start at zero: the kernels only OR flags into it
   if (cudaMemsetAsync(ws, 0, kStatusBytes, st) != cudaSuccess) return MLA_ERR_CUDA;
   if (launch_schedule_whole_tiles(seqlens, si, W, sched, static_cast<int32_t*>(ws), st) != cudaSuccess)
     return MLA_ERR_CUDA;
-  rc = launch_decode_sm100(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, ws, 0, out, lse,
-                           st);
+  rc = enqueue_decode_sm100(prep, shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, ws, 0,
+                            out, lse, st);
   if (rc != MLA_OK) return rc;
   if (launch_combine(sched, ws, out, lse, int(num_tiles), 0, st) != cudaSuccess) return MLA_ERR_CUDA;
   if (device_status && cudaMemcpyAsync(device_status, ws, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)

@@ -371,13 +371,7 @@ int proj_num_sms() {
 
 template <int KC>
 int launch_proj(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& o, ProjArgs a, cudaStream_t stream) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(proj_sm100_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(kProjSmem));
-  });
-  if (attr_err != cudaSuccess) return MLA_ERR_CUDA;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(&proj_sm100_kernel<KC>), int(kProjSmem))) return MLA_ERR_CUDA;
   const int sms = proj_num_sms();
   if (sms < 0) return MLA_ERR_CUDA;
   a.n_tiles = (a.rows + kTileN - 1) / kTileN;

@@ -20,7 +20,7 @@
 // run without partials, jagged ones are cut.
 #include <cuda_runtime.h>
 
-#include "common.cuh"
+#include "kernel_util.cuh"
 
 namespace mla {
 
@@ -456,12 +456,11 @@ size_t schedule_whole_tiles_smem(int num_tiles) {
 
 cudaError_t launch_schedule_whole_tiles(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
                                         int32_t* status, cudaStream_t stream) {
-  const size_t smem = size_t(s.batch) * s.tiles_per_req * 8;
-  if (smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(schedule_whole_tiles_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSchedSmemMax));
-    if (e != cudaSuccess) return e;
-  }
+  const size_t smem = schedule_whole_tiles_smem(s.batch * s.tiles_per_req);
+  if (smem == 0 && s.batch * s.tiles_per_req > 0) return cudaErrorInvalidValue;   // over the shared-memory budget
+  if (smem > 48 * 1024 &&
+      !ensure_smem_attr(reinterpret_cast<const void*>(&schedule_whole_tiles_kernel), int(kSchedSmemMax)))
+    return cudaErrorInvalidValue;
   schedule_whole_tiles_kernel<<<1, kSchedThreads, smem, stream>>>(seqlens, s, W, sched, status);
   return cudaGetLastError();
 }
@@ -470,11 +469,9 @@ cudaError_t launch_schedule(const int32_t* seqlens, const ShapeInfo& s, int W, i
                             cudaStream_t stream) {
   const size_t smem = sched_smem_bytes(s.batch * s.tiles_per_req, W);
   if (smem <= kSchedSmemMax) {
-    if (smem > 48 * 1024) {
-      const cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(kSchedSmemMax));
-      if (e != cudaSuccess) return e;
-    }
+    if (smem > 48 * 1024 &&
+        !ensure_smem_attr(reinterpret_cast<const void*>(&schedule_kernel), int(kSchedSmemMax)))
+      return cudaErrorInvalidValue;
     schedule_kernel<<<1, kSchedThreads, smem, stream>>>(seqlens, s, W, sched);
   } else {
     schedule_kernel_global<<<1, 32, 0, stream>>>(seqlens, s, W, sched);

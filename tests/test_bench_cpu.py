@@ -43,7 +43,7 @@ def test_bench_functions_load_only_defined_globals():
 def test_reference_arm_prints_its_json_line():
     out = subprocess.run(
         [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
-         "--ref-requests", "1"],
+         "--ref-seconds", "0.05"],
         cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     line = [l for l in out.stdout.splitlines() if l.startswith("{")][-1]
@@ -51,6 +51,10 @@ def test_reference_arm_prints_its_json_line():
     assert rec["impl"] == "reference"
     assert rec["value"] > 0 and rec["steps"] == 1 and rec["warmup"] == 0
     assert rec["config"]["workload"] == "dsv3_b64_h128_t4096_paged"
+    # the same config dict as the GPU arm prints for this workload
+    import mla_workloads as mw
+    b = _load_bench()
+    assert rec["config"] == json.loads(json.dumps(b.config_dict(mw.make_config(2, seed=0), 1)))
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
     assert rec["higher_is_better"] is True
@@ -70,7 +74,7 @@ def test_reference_arm_under_torchrun_two_ranks():
         [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
          "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
          os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
-         "--ref-requests", "1"],
+         "--ref-seconds", "0.05"],
         cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]

@@ -8,7 +8,7 @@ import torch
 import mla_latent_space_b200 as mla
 import mla_workloads as mw
 import oracle
-from gpu_helpers import (assert_parity, check_full, check_sampled, compare, run, shape_of, to_device)
+from gpu_helpers import (assert_parity, check_full, compare, run, shape_of, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -123,11 +123,44 @@ def test_bad_page_id_is_flagged_not_faulted():
     assert_parity(compare(O[:1], L[:1], O_ref[:1], L_ref[:1]), "unaffected request")
 
 
-# ---- the five workloads at full size, sampled rows -------------------------
+def test_value_beyond_fp16_range_is_flagged():
+    """PV runs in fp16: a bf16 value entry of 1e5 cannot be represented.
+    The decode flags it (MLA_ERR_DEVICE_CHECK) instead of returning a wrong
+    result silently; the request that does not read that page is still at
+    parity."""
+    wl = mw.make(2, 1, 128, [100, 100], seed=17, name="v_overflow")
+    page = int(wl.block_table[1, 0])
+    wl.pool[page, 5, 17] = 1e5                  # a value column (< 512) of request 1
+    O, L, st = run(wl)
+    assert st == -6                             # MLA_ERR_DEVICE_CHECK
+    O_ref, L_ref = oracle.decode(wl, rows=[(0, 0)])
+    assert_parity(compare(O[:1, 0], L[:1, 0], O_ref, L_ref), "unaffected request")
+
+
+def test_fp8_value_times_scale_beyond_fp16_range_is_flagged():
+    """The FP8 cache's values times their per-token scale enter PV as fp16:
+    a scale of 1e3 puts the token's larger e4m3 values above 65504."""
+    import dataclasses
+    wl = mw.make(2, 1, 128, [100, 100], cache_dtype="fp8", seed=18, name="fp8_v_overflow")
+    page = int(wl.block_table[1, 0])
+    ks = wl.kv_scale.clone()
+    ks[page, 9] = 1e3
+    wl = dataclasses.replace(wl, kv_scale=ks)
+    O, L, st = run(wl)
+    assert st == -6
+    O_ref, L_ref = oracle.decode(wl, rows=[(0, 0)])
+    assert_parity(compare(O[:1, 0], L[:1, 0], O_ref, L_ref), "unaffected request")
+
+
+# ---- the five workloads at full size, every row ------------------------------
 
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
-def test_full_size_configs_sampled(cfg):
-    check_sampled(mw.make_config(cfg), n=4)
+def test_full_size_configs_every_row(cfg):
+    """Configs 2-5 at their full sizes, the launch configuration the bench
+    times: every O element and every LSE of the batch against the oracle
+    (which gathers one request's cache at a time, so the 131072-token
+    requests of the jagged batch stay within a few hundred MB)."""
+    check_full(mw.make_config(cfg))
 
 
 # ---- FP8 cache: the kFp8 kernel across the same edge cases ------------------
