@@ -42,14 +42,15 @@ L2_FLUSH_BYTES = 256 << 20
 # for the kernel sources they were taken on: reported as null as soon as any
 # of them differs (checked by content hash at run time).
 TRAFFIC_SOURCES_SHA1 = {
-    "mla_latent_space_b200/csrc/decode_sm100.cu": "4fcb6e9d788f6c4d667bf4245664a7b4df75dc8b",
+    "mla_latent_space_b200/csrc/decode_sm100.cu": "b58f7f984c0a4e27f555c33c1e2cc1c2b72f5c47",
     "mla_latent_space_b200/csrc/sm100_ptx.cuh": "a666c6fb95adecc45850f281b1be3ecacba5d16c",
-    "mla_latent_space_b200/csrc/kernel_util.cuh": "c304dedb0965e65632e557168f97693bf2077cdb",
-    "mla_latent_space_b200/csrc/common.cuh": "1bda35f3e244dc99d70c2901283243f600e444f6",
+    "mla_latent_space_b200/csrc/kernel_util.cuh": "9d7c3e48c90d2d444145ab84159f8400e402f999",
+    "mla_latent_space_b200/csrc/common.cuh": "7c6e8d72ef32d67aafb386e65a6767fa77f51a7f",
+    "mla_latent_space_b200/csrc/decode_launch.cuh": "1ad27cf53b46b1c703e25fb308cac7eb7caaeece",
 }
 TRAFFIC_BYTES = {
-    "dsv3_b64_h128_t4096_paged": 311.547136e6 + 4.920576e6,
-    "fp8_b64_h128_t32768": 1374.59968e6 + 23.452416e6,
+    "dsv3_b64_h128_t4096_paged": 311557632 + 4642560,
+    "fp8_b64_h128_t32768": 1374624000 + 22552064,
 }
 
 
