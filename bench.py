@@ -623,18 +623,16 @@ def time_steps(args, dw, flush, K, world=1, local=0, sample_clocks=False):
     torch.cuda.synchronize()
     if clocks:
         clocks.start()
-    # the step is bracketed by events only at its ends: an event between two
-    # of its kernels would stop the next one from launching behind the
-    # previous (programmatic dependent launch)
+    # Each iteration runs the step twice: once bracketed by events only at
+    # its ends (an event between two of its kernels would stop the next one
+    # from launching behind the previous, programmatic dependent launch), and
+    # once with events around the decode launch alone, for the roofline.
+    # Interleaving them gives both the same clocks and power state.
     for k in range(K):
         flush.zero_()
         ev_step[k][0].record(stream)
         dw.step()
         ev_step[k][1].record(stream)
-    torch.cuda.synchronize()
-    # the decode kernel alone, for the roofline: the same steps with events
-    # around the decode launch
-    for k in range(K):
         flush.zero_()
         dw.step(ev_dec[k])
     torch.cuda.synchronize()
@@ -699,11 +697,11 @@ def per_config(args, dev, flush, pk, pk_kind, headline=None):
     K = max(5, min(args.steps, args.per_config_steps))
     for cfg in (1, 2, 3, 4, 5):
         if headline is not None and cfg == args.config:
-            wl, step_ms, dec_ms = headline
+            wl, step_ms, dec_ms, clk = headline
         else:
             wl = mw.make_config(cfg, seed=0)
             dw = DeviceWorkload(wl, dev)
-            step_ms, dec_ms, _ = time_steps(args, dw, flush, K)
+            step_ms, dec_ms, clk = time_steps(args, dw, flush, K, sample_clocks=True)
             del dw
             torch.cuda.empty_cache()
         flops, nbytes = cost.workload_cost(wl)
@@ -712,7 +710,7 @@ def per_config(args, dev, flush, pk, pk_kind, headline=None):
         ent = {"workload": wl.name, "steps": len(step_ms), "us_per_step": us,
                "tflops": flops / (us * 1e-6) / 1e12, "kv_gbs": nbytes / (us * 1e-6) / 1e9,
                "decode_us": dus, "flops": flops, "bytes": nbytes,
-               "roofline": roofline(wl, dus * 1e-3, pk, pk_kind, captured_traffic(wl.name))}
+               "roofline": roofline(wl, dus * 1e-3, pk, pk_kind, captured_traffic(wl.name)), "clocks": clk}
         if cfg == 1:
             ent["note"] = "0.66 MB and 18 MFLOP: launch-bound, reported only"
         if not args.no_cpu_baseline:
@@ -767,7 +765,7 @@ def run_ours(args, wl, world, rank, local):
     d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
     del dw
     torch.cuda.empty_cache()
-    pcfg, pc_launches = per_config(args, dev, flush, pk, pk_kind, headline=(wl, step_ms, dec_ms)) \
+    pcfg, pc_launches = per_config(args, dev, flush, pk, pk_kind, headline=(wl, step_ms, dec_ms, clk)) \
         if extras and not args.no_per_config else (None, 0)
 
     flops, nbytes = cost.workload_cost(wl)

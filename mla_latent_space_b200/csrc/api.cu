@@ -21,8 +21,6 @@ cudaError_t launch_decode_simt(const void* q, const void* kv, const float* kv_sc
                                float* lse, int num_pages, int fp8, int cap_slots, int grid_ctas,
                                cudaStream_t stream);
 #endif
-cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
-                           int cap_slots, cudaStream_t stream);
 cudaError_t launch_sparse_gather(const int32_t* indices, int topk, const int32_t* seqlens, int batch, int s_q,
                                  const int32_t* block_table, int max_pages, int num_pages, const void* pool,
                                  const float* kv_scale, void* scratch, float* vscale, int vpages, int32_t* vseqlens,
@@ -31,13 +29,13 @@ cudaError_t launch_var6_old_len(const int32_t* seqlens, int batch, int n_new, in
                                 cudaStream_t stream);
 cudaError_t launch_var6_new(const void* q, const void* k_new, const void* v_new, const void* pool, bool fp8,
                             const int32_t* block_table, const int32_t* seqlens, const void* o_old,
-                            const float* lse_old, int batch, int s_q, int heads, int n_new, int max_pages,
-                            int num_pages, int causal, float scale, void* out, float* lse, void* status_ws,
-                            cudaStream_t stream);
+                            const void* o_old_lo, const float* lse_old, int batch, int s_q, int heads, int n_new,
+                            int max_pages, int num_pages, int causal, float scale, void* out, float* lse,
+                            void* status_ws, cudaStream_t stream);
 int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* qz, int32_t* status,
                     cudaStream_t stream);
 int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
-                        cudaStream_t stream);
+                        cudaStream_t stream, const void* o_lat_lo = nullptr, void* out_lo = nullptr);
 }  // namespace mla
 
 using namespace mla;
@@ -167,11 +165,11 @@ bool sparse_layout(const mla_shape_t* s, int topk, int num_sms, SparseLayout* L)
 
 // Workspace of the MLAvar6+ split decode (every region 256-byte aligned):
 // the old lengths t - n, the schedule and decode workspace of the latent
-// part (a non-causal decode over the old tokens), its latent output and
-// lse, and its decompressed output.
+// part (a non-causal decode over the old tokens), its latent output (two
+// bf16 terms) and lse, and its decompressed output (two bf16 terms).
 struct Var6Layout {
   mla_shape_t oshape;
-  size_t oldlen, sched, sched_bytes, ws, ws_bytes, olat, lse_old, oold, total;
+  size_t oldlen, sched, sched_bytes, ws, ws_bytes, olat, olat_lo, lse_old, oold, oold_lo, total;
 };
 
 bool var6_layout(const mla_shape_t* s, int n_new, int num_sms, Var6Layout* L) {
@@ -193,9 +191,13 @@ bool var6_layout(const mla_shape_t* s, int n_new, int num_sms, Var6Layout* L) {
   off = up(off + L->ws_bytes);
   L->olat = off;
   off = up(off + rows * MLA_D_V * 2);
+  L->olat_lo = off;
+  off = up(off + rows * MLA_D_V * 2);
   L->lse_old = off;
   off = up(off + rows * 4);
   L->oold = off;
+  off = up(off + rows * MLA_D_HEAD * 2);
+  L->oold_lo = off;
   off = up(off + rows * MLA_D_HEAD * 2);
   L->total = off;
   return true;
@@ -388,8 +390,10 @@ int mla_var6_decode_fwd(const mla_shape_t* shape, int n_new, const void* qz, con
   void* sched = w + L.sched;
   void* ws = w + L.ws;
   void* olat = w + L.olat;
+  void* olat_lo = w + L.olat_lo;
   float* lse_old = reinterpret_cast<float*>(w + L.lse_old);
   void* oold = w + L.oold;
+  void* oold_lo = w + L.oold_lo;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int b = shape->batch, s = shape->s_q, h = shape->num_heads;
   if (launch_var6_old_len(seqlens, b, n_new, shape->max_pages_per_seq, oldlen, st) != cudaSuccess) return MLA_ERR_CUDA;
@@ -398,13 +402,13 @@ int mla_var6_decode_fwd(const mla_shape_t* shape, int n_new, const void* qz, con
     return MLA_ERR_CUDA;
   const int cap = cap_slots_for(L.ws_bytes);
   rc = launch_decode_sm100(&L.oshape, qz, kv_cache, kv_scale, block_table, oldlen, softmax_scale, sched, ws, cap, olat,
-                           lse_old, st);
+                           lse_old, st, olat_lo);
   if (rc != MLA_OK) return rc;
-  if (launch_combine(sched, ws, olat, lse_old, si.batch * si.tiles_per_req, cap, st) != cudaSuccess)
+  if (launch_combine(sched, ws, olat, lse_old, si.batch * si.tiles_per_req, cap, st, olat_lo) != cudaSuccess)
     return MLA_ERR_CUDA;
-  rc = launch_decompress_o(b * s, h, olat, w_kvb2, oold, static_cast<int32_t*>(ws), st);
+  rc = launch_decompress_o(b * s, h, olat, w_kvb2, oold, static_cast<int32_t*>(ws), st, olat_lo, oold_lo);
   if (rc != MLA_OK) return rc;
-  return launch_var6_new(q, k_new, v_new, kv_cache, fp8, block_table, seqlens, oold, lse_old, b, s, h, n_new,
+  return launch_var6_new(q, k_new, v_new, kv_cache, fp8, block_table, seqlens, oold, oold_lo, lse_old, b, s, h, n_new,
                          shape->max_pages_per_seq, shape->num_pages, shape->causal, softmax_scale, out, lse, ws,
                          st) == cudaSuccess
              ? MLA_OK

@@ -2,6 +2,7 @@
 // Piece i of a row carries its normalised partial output O_i and its lse_i;
 // the row's result is L = ln sum_i e^{lse_i} and O = sum_i e^{lse_i - L} O_i.
 // Tiles that no worker touched (no visible key) get O = 0 and lse = -inf.
+// With out_lo, O is written as two bf16 terms (out + out_lo).
 //
 // One warp per row, (tile, 16 row blocks) CTAs of 8 warps: the lanes read
 // the pieces' lse values at once and reduce max and sum with shuffles; then
@@ -9,6 +10,7 @@
 // loads in flight per lane).  At most 64 registers a thread, so that four
 // CTAs share an SM and every row of a typical batch is in flight in about
 // one wave: the kernel is bound by how many loads are outstanding.
+#include "decode_launch.cuh"
 #include "kernel_util.cuh"
 #include "sm100_ptx.cuh"
 
@@ -21,7 +23,7 @@ constexpr int kRowBlocks = MLA_TILE_ROWS / kWarps;   // 16
 
 __global__ void __launch_bounds__(kWarps * 32, 4)
 combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __nv_bfloat16* __restrict__ out,
-               float* __restrict__ lse, int cap_slots) {
+               __nv_bfloat16* __restrict__ out_lo, float* __restrict__ lse, int cap_slots) {
   ptx::griddep_wait();   // launched programmatically behind the decode kernel
   const SchedView sv(sched);
   void* ws = const_cast<void*>(ws_c);
@@ -40,9 +42,14 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
     return;
   }
   __nv_bfloat16* o = out + (size_t(r) * rows_total + rho) * MLA_D_V;
+  __nv_bfloat16* ol = out_lo != nullptr ? out_lo + (size_t(r) * rows_total + rho) * MLA_D_V : nullptr;
   if (n == 0) {
     reinterpret_cast<uint4*>(o)[lane * 2] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(o)[lane * 2 + 1] = make_uint4(0, 0, 0, 0);
+    if (ol != nullptr) {
+      reinterpret_cast<uint4*>(ol)[lane * 2] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(ol)[lane * 2 + 1] = make_uint4(0, 0, 0, 0);
+    }
     if (lane == 0) lse[size_t(r) * rows_total + rho] = -INFINITY;
     return;
   }
@@ -92,12 +99,20 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
   }
 #pragma unroll
   for (int c = 0; c < MLA_D_V / 128; ++c) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[c].x, acc[c].y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[c].z, acc[c].w);
+    const __nv_bfloat162 h01 = __floats2bfloat162_rn(acc[c].x, acc[c].y);
+    const __nv_bfloat162 h23 = __floats2bfloat162_rn(acc[c].z, acc[c].w);
     uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    pk.x = *reinterpret_cast<const uint32_t*>(&h01);
+    pk.y = *reinterpret_cast<const uint32_t*>(&h23);
     reinterpret_cast<uint2*>(o)[lane + 32 * c] = pk;
+    if (ol != nullptr) {   // second term: bf16 of what the first one dropped
+      const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+      const __nv_bfloat162 l01 = __floats2bfloat162_rn(acc[c].x - f01.x, acc[c].y - f01.y);
+      const __nv_bfloat162 l23 = __floats2bfloat162_rn(acc[c].z - f23.x, acc[c].w - f23.y);
+      pk.x = *reinterpret_cast<const uint32_t*>(&l01);
+      pk.y = *reinterpret_cast<const uint32_t*>(&l23);
+      reinterpret_cast<uint2*>(ol)[lane + 32 * c] = pk;
+    }
   }
   if (lane == 0) lse[size_t(r) * rows_total + rho] = L;
 }
@@ -105,7 +120,7 @@ combine_kernel(const void* __restrict__ sched, const void* __restrict__ ws_c, __
 }  // namespace
 
 cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
-                           int cap_slots, cudaStream_t stream) {
+                           int cap_slots, cudaStream_t stream, void* out_lo) {
   if (num_tiles == 0) return cudaSuccess;
   // programmatic dependent launch behind the decode kernel (the kernel waits
   // for it before reading anything)
@@ -119,8 +134,8 @@ cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, sched, ws, static_cast<__nv_bfloat16*>(out), lse,
-                                           cap_slots);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, sched, ws, static_cast<__nv_bfloat16*>(out),
+                                           static_cast<__nv_bfloat16*>(out_lo), lse, cap_slots);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -26,13 +26,23 @@ struct DecodePrepared {
 int prepare_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, DecodePrepared* pr);
 
 // Enqueues the decode kernel built by prepare_decode_sm100 on `stream`.
+// out_lo (optional, bf16 like out): whole tiles then write O as two terms,
+// out = bf16(O) and out_lo = bf16(O - out); split tiles leave both to the
+// combine (launch_combine with the same out_lo).
 int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, const void* q, const void* kv,
                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, float scale,
-                         const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
+                         const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream,
+                         void* out_lo = nullptr);
 
 // prepare + enqueue.
 int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
                         const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
-                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream);
+                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream,
+                        void* out_lo = nullptr);
+
+// The log-sum-exp merge of split tiles (and O = 0, lse = -inf for tiles
+// with no visible key); out_lo as for enqueue_decode_sm100.
+cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
+                           int cap_slots, cudaStream_t stream, void* out_lo = nullptr);
 
 }  // namespace mla

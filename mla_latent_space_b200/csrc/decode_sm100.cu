@@ -177,6 +177,7 @@ struct Params {
   const void* sched;
   void* ws;
   __nv_bfloat16* out;
+  __nv_bfloat16* out_lo;   // optional: out_lo = bf16(O - out), so out + out_lo carries O to ~2^-17
   float* lse;
   float scale_log2;   // softmax_scale * log2(e)
   int num_pages;
@@ -367,6 +368,16 @@ __device__ __forceinline__ void split_e4m3x4(uint32_t w01, uint32_t w23, float i
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// (a, b) -> bf16 pairs hi = (bf16(a), bf16(b)) and lo = bf16 of the
+// remainders (a - hi_a, b - hi_b; exact in fp32).
+__device__ __forceinline__ void split_bf16(float a, float b, uint32_t* hi, uint32_t* lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  *hi = *reinterpret_cast<const uint32_t*>(&h);
+  *lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
@@ -1098,7 +1109,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             tmem_ld32(tmem + lane_off + 32u * c, o);
             tmem_wait_ld();
             if (valid && slot_ok) {
-              if (whole) {
+              if (whole && p.out_lo == nullptr) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
                   dst_b[c * 4 + u] = make_uint4(
@@ -1106,6 +1117,20 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
                       pack_bf16(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv),
                       pack_bf16(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv),
                       pack_bf16(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv));
+              } else if (whole) {
+                // two-term output: hi = bf16(x), lo = bf16(x - hi)
+                uint4* dst_l =
+                    reinterpret_cast<uint4*>(p.out_lo + (size_t(r) * rows_total + (valid ? rho : 0)) * MLA_D_V);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  uint32_t hi[4], lo[4];
+#pragma unroll
+                  for (int k = 0; k < 4; ++k)
+                    split_bf16(__uint_as_float(o[8 * u + 2 * k]) * inv, __uint_as_float(o[8 * u + 2 * k + 1]) * inv,
+                               &hi[k], &lo[k]);
+                  dst_b[c * 4 + u] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                  dst_l[c * 4 + u] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
               } else {
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
@@ -1346,7 +1371,8 @@ int prepare_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv
 
 int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, const void* q, const void* kv,
                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, float scale,
-                         const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream) {
+                         const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream,
+                         void* out_lo) {
   Params prm;
   prm.q = static_cast<const uint16_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv);
@@ -1356,6 +1382,7 @@ int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, con
   prm.sched = sched;
   prm.ws = ws;
   prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.out_lo = static_cast<__nv_bfloat16*>(out_lo);
   prm.lse = lse;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.num_pages = shape->num_pages;
@@ -1383,12 +1410,12 @@ int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, con
 
 int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,
                         const int32_t* block_table, const int32_t* seqlens, float scale, const void* sched,
-                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream) {
+                        void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream, void* out_lo) {
   DecodePrepared pr;
   const int rc = prepare_decode_sm100(shape, q, kv, &pr);
   if (rc != MLA_OK) return rc;
   return enqueue_decode_sm100(pr, shape, q, kv, kv_scale, block_table, seqlens, scale, sched, ws, cap_slots, out,
-                              lse, stream);
+                              lse, stream, out_lo);
 }
 
 }  // namespace mla

@@ -14,8 +14,6 @@ namespace mla {
 size_t schedule_whole_tiles_smem(int num_tiles);
 cudaError_t launch_schedule_whole_tiles(const int32_t* seqlens, const ShapeInfo& s, int W, int32_t* sched,
                                         int32_t* status, cudaStream_t stream);
-cudaError_t launch_combine(const void* sched, const void* ws, void* out, float* lse, int num_tiles,
-                           int cap_slots, cudaStream_t stream);
 
 namespace {
 

@@ -80,6 +80,7 @@ struct ProjArgs {
   const uint8_t* rope_src;   // absorb: q, whose RoPE part is copied through; else null
   uint8_t* rope_dst;         // absorb: Qz
   int32_t* status;           // optional sticky status word
+  __nv_bfloat16* o_lo;       // two-term decompress: bf16 of what the bf16 output dropped
 };
 
 struct Unit {
@@ -141,10 +142,16 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 }
 
 // KC: number of 64-wide K chunks (absorb: d/64 = 2, decompress: 512/64 = 8).
-template <int KC>
+// kTwo: the activation comes as two bf16 terms (xmap + x2map, which carry an
+// fp32-accurate input) and the output goes out as two: D = (X + X2) . W^T is
+// one accumulation over 2 KC chunks (the weight chunks read twice), written
+// as o = bf16(D) through omap and o_lo = bf16(D - o) with plain stores.
+template <int KC, bool kTwo>
 __global__ void __launch_bounds__(kProjThreads, 1)
     proj_sm100_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
-                      const __grid_constant__ CUtensorMap omap, const ProjArgs a) {
+                      const __grid_constant__ CUtensorMap x2map, const __grid_constant__ CUtensorMap omap,
+                      const ProjArgs a) {
+  constexpr int KT = kTwo ? 2 * KC : KC;   // K chunks per unit
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full[kRing];
   __shared__ __align__(8) uint64_t empty[kRing];
@@ -175,6 +182,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&wmap);
     tma_prefetch_desc(&xmap);
+    if (kTwo) tma_prefetch_desc(&x2map);
     tma_prefetch_desc(&omap);
   }
   if (warp == 1) {
@@ -199,7 +207,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         const Unit x = unit_of(a, u);
         const int wy = x.head * a.w_rows_per_head + x.m0, xx = x.head * a.x_cols_per_head;
         bool go = true;
-        for (int kc = 0; kc < KC; ++kc, ++g) {
+        for (int kc = 0; kc < KT; ++kc, ++g) {
           const int s = g % kRing;
           const int fill = g / kRing;   // earlier fills of stage s
           if (fill > 0 && !wait_bounded(smem_u32(&empty[s]), uint32_t((fill - 1) & 1), abort, a.status)) {
@@ -207,9 +215,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             break;
           }
           const uint32_t st = base + uint32_t(s) * kStage;
+          const int kw = kc % KC;   // the weight chunk (read twice in two-term mode)
           mbar_arrive_expect_tx(smem_u32(&full[s]), kStage);
-          tma_load_2d(st, &wmap, 64 * kc, wy, smem_u32(&full[s]));
-          tma_load_2d(st + kChunk, &xmap, xx + 64 * kc, x.r0, smem_u32(&full[s]));
+          tma_load_2d(st, &wmap, 64 * kw, wy, smem_u32(&full[s]));
+          tma_load_2d(st + kChunk, (kTwo && kc >= KC) ? &x2map : &xmap, xx + 64 * kw, x.r0, smem_u32(&full[s]));
         }
         if (!go) break;
       }
@@ -233,7 +242,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(acc * kTileN);
         bool go = true;
-        for (int kc = 0; kc < KC; ++kc, ++g) {
+        for (int kc = 0; kc < KT; ++kc, ++g) {
           const int s = g % kRing;
           if (!wait_bounded(smem_u32(&full[s]), uint32_t((g / kRing) & 1), abort, a.status)) {
             go = false;
@@ -300,15 +309,27 @@ __global__ void __launch_bounds__(kProjThreads, 1)
           const uint32_t rowaddr = stg + uint32_t(j >> 1) * kStagingBox + uint32_t(row) * 128u;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
+            uint32_t w[4], wl[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const __nv_bfloat162 pr =
-                  __floats2bfloat162_rn(__uint_as_float(v[8 * c + 2 * k]), __uint_as_float(v[8 * c + 2 * k + 1]));
+              const float f0 = __uint_as_float(v[8 * c + 2 * k]), f1 = __uint_as_float(v[8 * c + 2 * k + 1]);
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(f0, f1);
               w[k] = *reinterpret_cast<const uint32_t*>(&pr);
+              if constexpr (kTwo) {
+                const float2 h = __bfloat1622float2(pr);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(f0 - h.x, f1 - h.y);
+                wl[k] = *reinterpret_cast<const uint32_t*>(&lo);
+              }
             }
             const uint32_t chunk = uint32_t(4 * (j & 1) + c);
             st_shared_v4(rowaddr + ((chunk ^ sw) << 4), w[0], w[1], w[2], w[3]);
+            if constexpr (kTwo) {
+              if (x.r0 + row < a.rows) {
+                __nv_bfloat16* dst = a.o_lo + (size_t(x.r0 + row) * a.heads * a.o_cols_per_head +
+                                               size_t(x.head) * a.o_cols_per_head + x.m0 + 32 * j + 8 * c);
+                *reinterpret_cast<uint4*>(dst) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+              }
+            }
           }
         }
       }
@@ -369,9 +390,11 @@ int proj_num_sms() {
   return n;
 }
 
-template <int KC>
-int launch_proj(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& o, ProjArgs a, cudaStream_t stream) {
-  if (!ensure_smem_attr(reinterpret_cast<const void*>(&proj_sm100_kernel<KC>), int(kProjSmem))) return MLA_ERR_CUDA;
+template <int KC, bool kTwo>
+int launch_proj(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& x2, const CUtensorMap& o, ProjArgs a,
+                cudaStream_t stream) {
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(&proj_sm100_kernel<KC, kTwo>), int(kProjSmem)))
+    return MLA_ERR_CUDA;
   const int sms = proj_num_sms();
   if (sms < 0) return MLA_ERR_CUDA;
   a.n_tiles = (a.rows + kTileN - 1) / kTileN;
@@ -387,7 +410,7 @@ int launch_proj(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& o
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, proj_sm100_kernel<KC>, w, x, o, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, proj_sm100_kernel<KC, kTwo>, w, x, x2, o, a);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -411,16 +434,22 @@ int launch_absorb_q(int rows, int heads, const void* q, const void* w_k, void* q
   a.rope_src = static_cast<const uint8_t*>(q);
   a.rope_dst = static_cast<uint8_t*>(qz);
   a.status = status;
+  a.o_lo = nullptr;
   a.m_tiles = MLA_D_V / kTileM;
-  return launch_proj<MLA_D_HEAD / 64>(w, x, o, a, stream);
+  return launch_proj<MLA_D_HEAD / 64, false>(w, x, x, o, a, stream);
 }
 
+// o_lat_lo / out_lo: both null (one-term bf16 decompression), or both set
+// (two-term: the input is o_lat + o_lat_lo, the output out + out_lo).
 int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kvb2, void* out, int32_t* status,
-                        cudaStream_t stream) {
-  CUtensorMap w, x, o;
+                        cudaStream_t stream, const void* o_lat_lo, void* out_lo) {
+  CUtensorMap w, x, x2, o;
   const uint64_t h = uint64_t(heads), R = uint64_t(rows);
+  const bool two = o_lat_lo != nullptr;
+  if (two != (out_lo != nullptr)) return MLA_ERR_INVALID_ARG;
   if (!make_map(&w, w_kvb2, MLA_D_V, h * MLA_D_HEAD, 2 * MLA_D_V)) return MLA_ERR_CUDA;
   if (!make_map(&x, o_lat, h * MLA_D_V, R, 2 * h * MLA_D_V)) return MLA_ERR_CUDA;
+  if (two && !make_map(&x2, o_lat_lo, h * MLA_D_V, R, 2 * h * MLA_D_V)) return MLA_ERR_CUDA;
   if (!make_map(&o, out, h * MLA_D_HEAD, R, 2 * h * MLA_D_HEAD)) return MLA_ERR_CUDA;
   ProjArgs a;
   a.w_rows_per_head = MLA_D_HEAD;
@@ -431,8 +460,10 @@ int launch_decompress_o(int rows, int heads, const void* o_lat, const void* w_kv
   a.rope_src = nullptr;
   a.rope_dst = nullptr;
   a.status = status;
+  a.o_lo = static_cast<__nv_bfloat16*>(out_lo);
   a.m_tiles = MLA_D_HEAD / kTileM;
-  return launch_proj<MLA_D_V / 64>(w, x, o, a, stream);
+  return two ? launch_proj<MLA_D_V / 64, true>(w, x, x2, o, a, stream)
+             : launch_proj<MLA_D_V / 64, false>(w, x, x, o, a, stream);
 }
 
 }  // namespace mla

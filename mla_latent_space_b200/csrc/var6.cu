@@ -8,7 +8,9 @@
 //   1. old lengths t - n (var6_old_len_kernel);
 //   2. the latent decode over the old tokens (schedule, tcgen05 decode,
 //      combine) and the output decompression of its result (the projection
-//      kernel), giving O_old [b, s, h, d] and lse_old;
+//      kernel), giving O_old [b, s, h, d] and lse_old.  Both intermediates
+//      travel as two bf16 terms (hi + lo, fp32-accurate), so the step adds
+//      no rounding of its own to the decode's;
 //   3. var6_new_kernel: attention of each (request, head)'s s query rows
 //      over its n decompressed tokens, merged with (O_old, lse_old).
 //
@@ -51,7 +53,8 @@ __global__ void __launch_bounds__(kVarThreads)
     var6_new_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
                     const uint16_t* __restrict__ v_new, const uint8_t* __restrict__ pool,
                     const int32_t* __restrict__ block_table, const int32_t* __restrict__ seqlens,
-                    const uint16_t* __restrict__ o_old, const float* __restrict__ lse_old, int s_q, int heads,
+                    const uint16_t* __restrict__ o_old, const uint16_t* __restrict__ o_old_lo,
+                    const float* __restrict__ lse_old, int s_q, int heads,
                     int n_new, int max_pages, int num_pages, int causal, float scale, __nv_bfloat16* __restrict__ out,
                     float* __restrict__ lse, void* status_ws) {
   constexpr int kQ = MLA_D_HEAD + MLA_D_ROPE;   // 192
@@ -221,10 +224,14 @@ __global__ void __launch_bounds__(kVarThreads)
       wo = so / (so + sn);
       wn = sn / (so + sn);
     }
+    // the old part arrives as two bf16 terms, hi + lo (fp32-accurate)
     const uint2 ob = *reinterpret_cast<const uint2*>(o_old + row * MLA_D_HEAD + 4 * lane);
+    const uint2 ol = *reinterpret_cast<const uint2*>(o_old_lo + row * MLA_D_HEAD + 4 * lane);
     const float inv = l_run[k] > 0.f ? 1.f / l_run[k] : 0.f;
-    const float o0 = wo * bf16_lo(ob.x) + wn * acc[k][0] * inv, o1 = wo * bf16_hi(ob.x) + wn * acc[k][1] * inv;
-    const float o2 = wo * bf16_lo(ob.y) + wn * acc[k][2] * inv, o3 = wo * bf16_hi(ob.y) + wn * acc[k][3] * inv;
+    const float a0 = bf16_lo(ob.x) + bf16_lo(ol.x), a1 = bf16_hi(ob.x) + bf16_hi(ol.x);
+    const float a2 = bf16_lo(ob.y) + bf16_lo(ol.y), a3 = bf16_hi(ob.y) + bf16_hi(ol.y);
+    const float o0 = wo * a0 + wn * acc[k][0] * inv, o1 = wo * a1 + wn * acc[k][1] * inv;
+    const float o2 = wo * a2 + wn * acc[k][2] * inv, o3 = wo * a3 + wn * acc[k][3] * inv;
     __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + row * MLA_D_HEAD + 4 * lane);
     dst[0] = __floats2bfloat162_rn(o0, o1);
     dst[1] = __floats2bfloat162_rn(o2, o3);
@@ -243,23 +250,24 @@ cudaError_t launch_var6_old_len(const int32_t* seqlens, int batch, int n_new, in
 
 cudaError_t launch_var6_new(const void* q, const void* k_new, const void* v_new, const void* pool, bool fp8,
                             const int32_t* block_table, const int32_t* seqlens, const void* o_old,
-                            const float* lse_old, int batch, int s_q, int heads, int n_new, int max_pages,
-                            int num_pages, int causal, float scale, void* out, float* lse, void* status_ws,
-                            cudaStream_t stream) {
+                            const void* o_old_lo, const float* lse_old, int batch, int s_q, int heads, int n_new,
+                            int max_pages, int num_pages, int causal, float scale, void* out, float* lse,
+                            void* status_ws, cudaStream_t stream) {
   const dim3 grid = dim3(unsigned(batch), unsigned(heads), 1u);
   const uint16_t* qq = static_cast<const uint16_t*>(q);
   const uint16_t* kk = static_cast<const uint16_t*>(k_new);
   const uint16_t* vv = static_cast<const uint16_t*>(v_new);
   const uint8_t* pp = static_cast<const uint8_t*>(pool);
   const uint16_t* oo = static_cast<const uint16_t*>(o_old);
+  const uint16_t* ool = static_cast<const uint16_t*>(o_old_lo);
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out);
   if (fp8)
-    var6_new_kernel<true><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, lse_old, s_q,
-                                                            heads, n_new, max_pages, num_pages, causal, scale, dst,
+    var6_new_kernel<true><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, ool, lse_old,
+                                                            s_q, heads, n_new, max_pages, num_pages, causal, scale, dst,
                                                             lse, status_ws);
   else
-    var6_new_kernel<false><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, lse_old, s_q,
-                                                             heads, n_new, max_pages, num_pages, causal, scale, dst,
+    var6_new_kernel<false><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, ool, lse_old,
+                                                             s_q, heads, n_new, max_pages, num_pages, causal, scale, dst,
                                                              lse, status_ws);
   return cudaGetLastError();
 }

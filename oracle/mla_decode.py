@@ -330,7 +330,7 @@ def new_token_attention(wl, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,
 
 
 def mlavar6_decode(wl, qz: np.ndarray, q: np.ndarray, k_new: np.ndarray, v_new: np.ndarray,
-                   w_kvb2: np.ndarray, n_new: int):
+                   w_kvb2: np.ndarray, n_new: int, rows=None):
     """Split latent + decompressed attention (page "MLA Cost Analysis &
     Regime Guide", "MLAvar6+ Design"), in float64.
 
@@ -344,33 +344,39 @@ def mlavar6_decode(wl, qz: np.ndarray, q: np.ndarray, k_new: np.ndarray, v_new: 
     Token positions: old j < t - n, new m at position t - n + m (m with a
     negative position, when t < n, does not exist); query i sees positions
     below visible_len(t, s, i, causal).
+    ``rows`` optionally lists (r, i) query tokens; the result then has shape
+    [len(rows), h, d] / [len(rows), h].
     Returns (out [b, s, h, d], lse [b, s, h])."""
     b, s, h, _ = qz.shape
     d = D_HEAD
-    out = np.zeros((b, s, h, d))
-    lse = np.zeros((b, s, h))
-    for r in range(b):
+    sel = [(r, i) for r in range(b) for i in range(s)] if rows is None else list(rows)
+    out = np.zeros((len(sel), h, d))
+    lse = np.zeros((len(sel), h))
+    C, C_r = None, -1
+    for n_sel, (r, i) in enumerate(sel):
         t = int(wl.seqlens[r])
-        C = gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale)
+        if r != C_r:
+            C, C_r = gather_rows(wl.pool, wl.block_table, r, t, wl.kv_scale), r
         o = max(t - n_new, 0)
-        for i in range(s):
-            Lv = max(visible_len(t, s, i, wl.causal), 0)
-            jo = min(o, Lv)                                   # visible old tokens
-            ms = np.arange(n_new)
-            pos = t - n_new + ms
-            keep = (pos >= 0) & (pos < Lv)                    # visible new tokens
-            ms, pos = ms[keep], pos[keep]
-            for hh in range(h):
-                x_old = wl.softmax_scale * (C[:jo] @ qz[r, i, hh])
-                x_new = wl.softmax_scale * (k_new[r, ms, hh] @ q[r, i, hh, :d] + C[pos, D_V:] @ q[r, i, hh, d:])
-                x = np.concatenate([x_old, x_new])
-                if x.size == 0:
-                    lse[r, i, hh] = -np.inf
-                    continue
-                m = x.max()
-                z = np.exp(x - m).sum()
-                lse[r, i, hh] = m + math.log(z)
-                w = np.exp(x - lse[r, i, hh])
-                vals = np.concatenate([C[:jo, :D_V] @ w_kvb2[hh].T, v_new[r, ms, hh]])
-                out[r, i, hh] = w @ vals
+        Lv = max(visible_len(t, s, i, wl.causal), 0)
+        jo = min(o, Lv)                                   # visible old tokens
+        ms = np.arange(n_new)
+        pos = t - n_new + ms
+        keep = (pos >= 0) & (pos < Lv)                    # visible new tokens
+        ms, pos = ms[keep], pos[keep]
+        for hh in range(h):
+            x_old = wl.softmax_scale * (C[:jo] @ qz[r, i, hh])
+            x_new = wl.softmax_scale * (k_new[r, ms, hh] @ q[r, i, hh, :d] + C[pos, D_V:] @ q[r, i, hh, d:])
+            x = np.concatenate([x_old, x_new])
+            if x.size == 0:
+                lse[n_sel, hh] = -np.inf
+                continue
+            m = x.max()
+            z = np.exp(x - m).sum()
+            lse[n_sel, hh] = m + math.log(z)
+            w = np.exp(x - lse[n_sel, hh])
+            vals = np.concatenate([C[:jo, :D_V] @ w_kvb2[hh].T, v_new[r, ms, hh]])
+            out[n_sel, hh] = w @ vals
+    if rows is None:
+        return out.reshape(b, s, h, d), lse.reshape(b, s, h)
     return out, lse

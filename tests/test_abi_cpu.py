@@ -130,11 +130,12 @@ def test_sparse_workspace_and_argument_checks():
 def test_var6_workspace_and_argument_checks():
     L = mla.lib()
     s = mla.make_shape(32, 16, 128, 64, 2048, causal=True)
-    # old lengths, schedule, decode workspace, then the latent output (bf16 x 512), its lse (fp32) and its
-    # decompression (bf16 x 128) for 32 x 16 x 128 rows
+    # old lengths, schedule, decode workspace, then the latent output (two bf16 terms x 512), its lse (fp32)
+    # and its decompression (two bf16 terms x 128) for 32 x 16 x 128 rows
     rows = 32 * 16 * 128
+    per_row = 2 * 1024 + 4 + 2 * 256
     nb = L.mla_var6_workspace_bytes(ctypes.byref(s), 64, 148)
-    assert rows * (1024 + 4 + 256) < nb < rows * (1024 + 4 + 256) + (64 << 20)
+    assert rows * per_row < nb < rows * per_row + (64 << 20)
     assert L.mla_var6_workspace_bytes(ctypes.byref(s), 8, 148) == 0          # causal needs n >= s_q
     assert L.mla_var6_workspace_bytes(ctypes.byref(mla.make_shape(32, 16, 128, 64, 2048)), 8, 148) > 0
     assert L.mla_var6_workspace_bytes(ctypes.byref(mla.make_shape(2, 33, 128, 64, 2048)), 64, 148) == 0
