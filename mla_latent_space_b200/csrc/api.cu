@@ -268,6 +268,24 @@ int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_
 }
 #endif
 
+#ifdef MLA_TEST_ENTRY_POINTS
+// Test-only entry point: mla_decode_fwd with the kernel's stall hook set, so
+// that one bounded wait runs out (after about 2 s) and the abort path runs.
+int mla_test_decode_stalled(const mla_shape_t* shape, const void* q, const void* kv_cache, const float* kv_scale,
+                            const int32_t* block_table, const int32_t* seqlens, float softmax_scale,
+                            const void* sched, void* workspace, size_t workspace_bytes, void* out, float* lse,
+                            void* stream) {
+  int rc = check_decode_args(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                             workspace_bytes, out, lse);
+  if (rc != MLA_OK) return rc;
+  DecodePrepared prep;
+  if ((rc = prepare_decode_sm100(shape, q, kv_cache, &prep)) != MLA_OK) return rc;
+  return enqueue_decode_sm100(prep, shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched,
+                              workspace, cap_slots_for(workspace_bytes), out, lse, static_cast<cudaStream_t>(stream),
+                              nullptr, 1);
+}
+#endif
+
 int mla_combine(const mla_shape_t* shape, const void* sched, const void* workspace, size_t workspace_bytes,
                 void* out, float* lse, void* stream) {
   int rc = check_shape(shape);

@@ -29,10 +29,12 @@ int prepare_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv
 // out_lo (optional, bf16 like out): whole tiles then write O as two terms,
 // out = bf16(O) and out_lo = bf16(O - out); split tiles leave both to the
 // combine (launch_combine with the same out_lo).
+// test_stall: 0, except from the test library's stalled-decode entry point
+// (a bounded wait in the kernel then runs out on purpose).
 int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, const void* q, const void* kv,
                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, float scale,
                          const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream,
-                         void* out_lo = nullptr);
+                         void* out_lo = nullptr, int test_stall = 0);
 
 // prepare + enqueue.
 int launch_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv, const float* kv_scale,

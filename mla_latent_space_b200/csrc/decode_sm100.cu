@@ -110,6 +110,7 @@ struct Bars {
   // score CTA (FP8 cache: also the query RoPE buffer)
   uint64_t z_full[kNZMax], z_empty[kNZMax], s_full, s_empty, q_ready, x_free[NX];
   uint64_t qpe_full, qpe_empty;
+  uint64_t never;   // test hook: a barrier nothing arrives on (Params::test_stall)
   // output CTA
   uint64_t v_loaded[NV], v_full[NV], pv_done[NV], p_full[NX], corr_go, corr_done, pv_blk[NB], o_free;
   // correction events, from the PV issuer warp to the correction warpgroup:
@@ -183,6 +184,7 @@ struct Params {
   int num_pages;
   int cap_slots;
   int q_rows;         // batch * s_q * heads
+  int test_stall;     // test hook, 0 in every product call (see the QK issuer)
 };
 
 
@@ -467,6 +469,7 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
     for (int s = 0; s < NB; ++s) mbar_init(bar(bars->pv_blk[s]), 1);
     mbar_init(bar(bars->qpe_full), 1);
     mbar_init(bar(bars->qpe_empty), 1);
+    mbar_init(bar(bars->never), 1);
     mbar_init(bar(bars->o_free), 128);
     mbar_init(bar(bars->mma_done), 1);
     bars->abort = 0;
@@ -640,6 +643,10 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
       const uint64_t qdesc = sdesc(sbase + L::qpe, 16, 1024);
       uint32_t zc = 0, bc = 0, pieces = 0;
       each_piece(sv, [&](const Piece& pc) {
+        // test hook (set only by the test library's stalled-decode entry
+        // point): a wait on a barrier nothing arrives on runs out, and the
+        // abort path (status bit, peer abort, drains, TMEM freed) runs
+        if (p.test_stall && !ewait(ctl, bar(bars->never), 0)) return false;
         // FP8 cache: the ring is shorter than the query, so its stages are
         // released one by one.  This warp walks every stage of the ring in
         // order (a parity wait is only sound when the stage's previous use
@@ -1372,7 +1379,7 @@ int prepare_decode_sm100(const mla_shape_t* shape, const void* q, const void* kv
 int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, const void* q, const void* kv,
                          const float* kv_scale, const int32_t* block_table, const int32_t* seqlens, float scale,
                          const void* sched, void* ws, int cap_slots, void* out, float* lse, cudaStream_t stream,
-                         void* out_lo) {
+                         void* out_lo, int test_stall) {
   Params prm;
   prm.q = static_cast<const uint16_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv);
@@ -1388,6 +1395,7 @@ int enqueue_decode_sm100(const DecodePrepared& pr, const mla_shape_t* shape, con
   prm.num_pages = shape->num_pages;
   prm.cap_slots = cap_slots;
   prm.q_rows = shape->batch * shape->s_q * shape->num_heads;
+  prm.test_stall = test_stall;
   const int clusters = pr.sms / 2 > 0 ? pr.sms / 2 : 1;
   // programmatic dependent launch: the prologue (barriers, TMEM, descriptor
   // prefetch) overlaps the scheduler kernel; the kernel waits for it before

@@ -19,6 +19,17 @@ int mla_decode_fwd_simt(const mla_shape_t* shape, const void* q, const void* kv_
                         void* workspace, size_t workspace_bytes, void* out, float* lse,
                         void* stream);
 
+/* mla_decode_fwd with the decode kernel's test hook set: one of its bounded
+ * waits waits on a barrier that nothing arrives on, runs out after about
+ * 2 s, and the kernel's abort path runs (status bit, both CTAs stop, copies
+ * and MMAs drained, tensor memory freed).  mla_get_device_status then
+ * reports MLA_ERR_TIMEOUT; the outputs are not valid.  Faults nothing. */
+int mla_test_decode_stalled(const mla_shape_t* shape, const void* q, const void* kv_cache,
+                            const float* kv_scale, const int32_t* block_table,
+                            const int32_t* seqlens, float softmax_scale, const void* sched,
+                            void* workspace, size_t workspace_bytes, void* out, float* lse,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,11 +23,9 @@ LSE_MAX_ABS = 1e-3
 _test_lib = None
 
 
-def mla_decode_fwd_simt(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace, out,
-                        lse, stream=None):
-    """The SIMT decode kernel of the test library (libmla_b200_test.so,
-    entry point declared in csrc/test_entry.h), same arguments as
-    mla.mla_decode_fwd."""
+def test_lib():
+    """The test library (libmla_b200_test.so): the product's objects plus the
+    entry points declared in csrc/test_entry.h."""
     global _test_lib
     if _test_lib is None:
         path = os.path.join(os.path.dirname(mla.LIB_PATH), "libmla_b200_test.so")
@@ -35,11 +33,26 @@ def mla_decode_fwd_simt(shape, q, kv_cache, kv_scale, block_table, seqlens, soft
             raise RuntimeError(f"{path} is missing: build it with `python -m mla_latent_space_b200.build`")
         L = ctypes.CDLL(path)
         vp, sz, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
-        L.mla_decode_fwd_simt.argtypes = [ctypes.POINTER(mla.mla_shape_t), vp, vp, vp, vp, vp, f32, vp, vp, sz,
-                                          vp, vp, vp]
-        L.mla_decode_fwd_simt.restype = ctypes.c_int
+        dec = [ctypes.POINTER(mla.mla_shape_t), vp, vp, vp, vp, vp, f32, vp, vp, sz, vp, vp, vp]
+        for name in ("mla_decode_fwd_simt", "mla_test_decode_stalled"):
+            getattr(L, name).argtypes = dec
+            getattr(L, name).restype = ctypes.c_int
         _test_lib = L
-    mla._decode_common(_test_lib.mla_decode_fwd_simt, "mla_decode_fwd_simt", shape, q, kv_cache, kv_scale,
+    return _test_lib
+
+
+def mla_decode_fwd_simt(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace, out,
+                        lse, stream=None):
+    """The SIMT decode kernel of the test library, same arguments as
+    mla.mla_decode_fwd."""
+    mla._decode_common(test_lib().mla_decode_fwd_simt, "mla_decode_fwd_simt", shape, q, kv_cache, kv_scale,
+                       block_table, seqlens, softmax_scale, sched, workspace, out, lse, stream)
+
+
+def mla_test_decode_stalled(shape, q, kv_cache, kv_scale, block_table, seqlens, softmax_scale, sched, workspace,
+                            out, lse, stream=None):
+    """mla_decode_fwd with the kernel's stall hook: one bounded wait runs out."""
+    mla._decode_common(test_lib().mla_test_decode_stalled, "mla_test_decode_stalled", shape, q, kv_cache, kv_scale,
                        block_table, seqlens, softmax_scale, sched, workspace, out, lse, stream)
 
 

@@ -8,7 +8,8 @@ import torch
 import mla_latent_space_b200 as mla
 import mla_workloads as mw
 import oracle
-from gpu_helpers import (assert_parity, check_full, compare, run, shape_of, to_device)
+from gpu_helpers import (assert_parity, check_full, compare, mla_test_decode_stalled, run, shape_of,
+                         to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -121,6 +122,32 @@ def test_bad_page_id_is_flagged_not_faulted():
     assert st == -6                         # MLA_ERR_DEVICE_CHECK
     O_ref, L_ref = oracle.decode(mw.make(2, 1, 128, [100, 100], seed=12))
     assert_parity(compare(O[:1], L[:1], O_ref[:1], L_ref[:1]), "unaffected request")
+
+
+def test_bounded_wait_runs_out_and_the_context_stays_usable():
+    """Failure detection without a fault: the test library's stalled decode
+    makes one of the kernel's bounded waits wait on a barrier that nothing
+    arrives on.  After its 2 s limit the kernel reports MLA_ERR_TIMEOUT
+    through the status word, both CTAs of every pair stop, drain and free
+    their tensor memory, and the next decode on the same context is at
+    parity."""
+    import time
+    wl = mw.make(2, 1, 128, [300, 100], seed=19, name="stall")
+    dev = to_device(wl)
+    shape = shape_of(wl)
+    dec = mla.Decoder(shape)
+    out = torch.empty((2, 1, 128, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((2, 1, 128), dtype=torch.float32, device="cuda")
+    dec.schedule(dev["seqlens"])
+    t0 = time.perf_counter()
+    mla_test_decode_stalled(shape, dev["q"], dev["pool"], None, dev["block_table"], dev["seqlens"], wl.softmax_scale,
+                            dec.sched, dec.workspace, out, lse)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert dec.status() == -5                       # MLA_ERR_TIMEOUT
+    assert 1.0 < dt < 30.0, dt                      # the wait's own limit ended it
+    assert dec.status() == 0                        # reading the status cleared it
+    check_full(wl)                                  # the context is still usable
 
 
 def test_value_beyond_fp16_range_is_flagged():
