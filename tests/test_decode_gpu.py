@@ -54,6 +54,29 @@ def test_simt_debug_path_matches_oracle():
     check_full(mw.make(2, 16, 128, [100, 300], causal=True, seed=8), simt=True)
 
 
+@pytest.mark.parametrize("h,s_q", [(1, 1), (3, 5), (128, 32), (256, 1)])
+def test_degenerate_and_large_tile_shapes(h, s_q):
+    """One head (a tile of one row), head counts that do not divide a tile,
+    32 query tokens (a causal step of 4096 rows per request), and 256 heads
+    (two tiles per query token)."""
+    check_full(mw.make(2, s_q, h, [max(s_q, 70), max(s_q, 300)], causal=s_q > 1, seed=26, name=f"shape_h{h}s{s_q}"))
+
+
+def test_many_short_requests():
+    """Far more tiles than SM pairs (600 requests of 1..200 tokens): the
+    scheduler packs many whole tiles per worker."""
+    rng = np.random.default_rng(27)
+    check_full(mw.make(600, 1, 128, rng.integers(1, 201, size=600).tolist(), seed=27, name="many_short"))
+
+
+def test_every_request_empty():
+    """No visible key anywhere: every O row is 0 and every lse is -inf."""
+    wl = mw.make(3, 2, 128, [0, 0, 0], seed=28, name="all_empty")
+    O, L, st = run(wl)
+    assert st == 0
+    assert np.all(O == 0) and np.all(np.isneginf(L))
+
+
 @pytest.mark.parametrize("n_sms", [2, 16, 148, 1000])
 def test_split_counts_agree(n_sms):
     # the same rows, cut into 1 .. hundreds of pieces, stay within tolerance
