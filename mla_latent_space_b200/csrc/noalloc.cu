@@ -4,6 +4,7 @@
 // most kNoAllocMaxTiles tiles; the schedule assigns whole tiles to workers
 // (schedule_whole_tiles_kernel), so no fp32 partial slot is ever needed.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <mutex>
 
@@ -25,6 +26,14 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// NVTX range around the call's host work (as for the other entry points).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // Address of this device's scratch and its SM count, looked up once per
 // device (the first call on a device, which therefore must not be made while
@@ -60,6 +69,7 @@ extern "C" int mla_decode_fwd_noalloc(const mla_shape_t* shape, const void* q, c
                                       const float* kv_scale, const int32_t* block_table, const int32_t* seqlens,
                                       float softmax_scale, void* out, float* lse, int32_t* device_status,
                                       void* stream) {
+  CallRange range_("mla_decode_fwd_noalloc");
   if (!shape) return MLA_ERR_INVALID_ARG;
   if (shape->batch < 1 || shape->s_q < 1 || shape->num_heads < 1 || shape->max_pages_per_seq < 1 ||
       shape->num_pages < 1)
