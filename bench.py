@@ -782,7 +782,9 @@ def run_ours(args, wl, world, rank, local):
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers"},
-            "gpu_launches": 3 * K}
+            "gpu_launches": 6 * K,
+            "gpu_launches_note": "schedule + decode + combine, twice per timed iteration (the step timed whole, "
+                                 "then with events around the decode launch)"}
     if pcfg is not None:
         line["per_config"] = pcfg
     if proj is not None:
