@@ -84,13 +84,15 @@ def peaks():
 
 class ClockSampler:
     """SM clock, power and clock-event reasons of this process's GPU, sampled
-    every 10 ms through NVML on a background thread while the timed region
-    runs (nvidia-smi's own loop is too coarse for a region of a second)."""
+    through NVML while the timed region runs: once as it starts, every 2 ms
+    on a background thread, and once as it ends, so that even a region of a
+    few milliseconds has several samples (nvidia-smi's own loop is too
+    coarse for that)."""
 
     REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
                ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"))
 
-    def __init__(self, cuda_index: int, period_s: float = 0.01):
+    def __init__(self, cuda_index: int, period_s: float = 0.002):
         self.cuda_index, self.period = cuda_index, period_s
         self.samples, self.reasons, self.power = [], set(), []
         self.max_mhz, self.err = None, None
@@ -123,19 +125,23 @@ class ClockSampler:
             return
         self._stop = threading.Event()
 
-        def loop():
-            while not self._stop.is_set():
-                try:
-                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
-                    self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
-                    r = int(get_reasons(h)) if get_reasons else 0
-                    for name, bit in bits.items():
-                        if bit and r & bit:
-                            self.reasons.add(name)
-                except Exception:
-                    pass
-                self._stop.wait(self.period)
+        def sample():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                self.power.append(nv.nvmlDeviceGetPowerUsage(h) / 1000.0)
+                r = int(get_reasons(h)) if get_reasons else 0
+                for name, bit in bits.items():
+                    if bit and r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
 
+        def loop():
+            while not self._stop.wait(self.period):
+                sample()
+
+        self._sample = sample
+        sample()
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
 
@@ -144,6 +150,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "not sampled"], "samples": 0}
         self._stop.set()
         self._thread.join(timeout=5)
+        self._sample()
         try:
             self._nvml.nvmlShutdown()
         except Exception:
@@ -151,7 +158,7 @@ class ClockSampler:
         sm = self.samples
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(sm),
-                "power_w_max": max(self.power) if self.power else None, "source": "nvml, 10 ms"}
+                "power_w_max": max(self.power) if self.power else None, "source": "nvml, 2 ms"}
 
 
 def dist_setup(n_gpus):
