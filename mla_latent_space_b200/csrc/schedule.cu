@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "kernel_util.cuh"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 
@@ -145,6 +146,9 @@ MLA_HD size_t sched_smem_bytes(int num_tiles, int W) {
 
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t* __restrict__ sched) {
+  // the decode kernel behind this one (a programmatic dependent) may start
+  // its prologue now; it reads the schedule only after this grid completes
+  ptx::griddep_launch_dependents();
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int64_t warp_tot[kSchedWarps];
   __shared__ int32_t flag_sh;
@@ -369,6 +373,7 @@ namespace {
 // sequential planner on the global copies (slow, but only for batches of
 // tens of thousands of tiles).
 __global__ void schedule_kernel_global(const int32_t* seqlens, ShapeInfo s, int W, int32_t* sched) {
+  ptx::griddep_launch_dependents();   // as in schedule_kernel
   if (threadIdx.x == 0 && blockIdx.x == 0) plan_schedule_seq(seqlens, s, W, sched);
 }
 }  // namespace
@@ -385,6 +390,7 @@ namespace {
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_whole_tiles_kernel(const int32_t* __restrict__ seqlens, ShapeInfo s, int W, int32_t* __restrict__ sched,
                             int32_t* __restrict__ status) {
+  ptx::griddep_launch_dependents();   // as in schedule_kernel
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int64_t warp_tot[kSchedWarps];
   __shared__ int32_t flag_sh;
