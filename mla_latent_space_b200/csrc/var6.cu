@@ -23,6 +23,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "kernel_util.cuh"
 
 namespace mla {
@@ -31,7 +33,7 @@ namespace {
 
 constexpr int kVarThreads = 128;
 constexpr int kVarWarps = kVarThreads / 32;
-constexpr int kMaxRowsPerWarp = 8;               // s_q <= 32
+constexpr int kMaxRowsPerWarp = 8;               // s_q <= 32 (query rows per warp, at most)
 constexpr int kChunk = 32;                       // new tokens per stage
 
 __global__ void var6_old_len_kernel(const int32_t* __restrict__ seqlens, int batch, int n_new, int cap,
@@ -47,9 +49,11 @@ __global__ void var6_old_len_kernel(const int32_t* __restrict__ seqlens, int bat
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// grid (batch, heads), 128 threads.
-template <bool kFp8>
-__global__ void __launch_bounds__(kVarThreads)
+// grid (batch, heads), 128 threads.  RPW: query rows per warp, the
+// smallest power of two >= ceil(s_q / 4), so that no row loop issues work
+// for rows that do not exist.
+template <bool kFp8, int RPW>
+__global__ void __launch_bounds__(kVarThreads, 4)
     var6_new_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k_new,
                     const uint16_t* __restrict__ v_new, const uint8_t* __restrict__ pool,
                     const int32_t* __restrict__ block_table, const int32_t* __restrict__ seqlens,
@@ -88,9 +92,9 @@ __global__ void __launch_bounds__(kVarThreads)
     }
   }
 
-  float m_run[kMaxRowsPerWarp], l_run[kMaxRowsPerWarp], acc[kMaxRowsPerWarp][4];
+  float m_run[RPW], l_run[RPW], acc[RPW][4];
 #pragma unroll
-  for (int k = 0; k < kMaxRowsPerWarp; ++k) {
+  for (int k = 0; k < RPW; ++k) {
     m_run[k] = -INFINITY;
     l_run[k] = 0.f;
     acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
@@ -162,22 +166,22 @@ __global__ void __launch_bounds__(kVarThreads)
     // every key word read from shared memory serves all of the warp's rows
     const int p = pos_s[lane];
     const int nrows = s_q > warp ? (s_q - warp + kVarWarps - 1) / kVarWarps : 0;
-    float xs[kMaxRowsPerWarp];
+    float xs[RPW];
 #pragma unroll
-    for (int k = 0; k < kMaxRowsPerWarp; ++k) xs[k] = 0.f;
+    for (int k = 0; k < RPW; ++k) xs[k] = 0.f;
 #pragma unroll 4
     for (int c = 0; c < kQ / 2; ++c) {
       const uint32_t kw = ks[lane][c];
       const float k0 = bf16_lo(kw), k1 = bf16_hi(kw);
 #pragma unroll
-      for (int k = 0; k < kMaxRowsPerWarp; ++k)
+      for (int k = 0; k < RPW; ++k)
         if (k < nrows) {
           const float2 qv = *reinterpret_cast<const float2*>(&qs[warp + kVarWarps * k][2 * c]);
           xs[k] = fmaf(qv.x, k0, fmaf(qv.y, k1, xs[k]));
         }
     }
 #pragma unroll
-    for (int k = 0; k < kMaxRowsPerWarp; ++k) {
+    for (int k = 0; k < RPW; ++k) {
       const int i = warp + kVarWarps * k;
       if (i >= s_q) break;
       const int vis = causal ? t - s_q + i + 1 : t;
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kVarThreads)
 
   // merge with the old tokens' result: L = ln(e^lse_old + e^lse_new)
 #pragma unroll
-  for (int k = 0; k < kMaxRowsPerWarp; ++k) {
+  for (int k = 0; k < RPW; ++k) {
     const int i = warp + kVarWarps * k;
     if (i >= s_q) break;
     const size_t row = (size_t(r) * s_q + i) * heads + hd;
@@ -261,14 +265,20 @@ cudaError_t launch_var6_new(const void* q, const void* k_new, const void* v_new,
   const uint16_t* oo = static_cast<const uint16_t*>(o_old);
   const uint16_t* ool = static_cast<const uint16_t*>(o_old_lo);
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out);
-  if (fp8)
-    var6_new_kernel<true><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, ool, lse_old,
-                                                            s_q, heads, n_new, max_pages, num_pages, causal, scale, dst,
-                                                            lse, status_ws);
-  else
-    var6_new_kernel<false><<<grid, kVarThreads, 0, stream>>>(qq, kk, vv, pp, block_table, seqlens, oo, ool, lse_old,
-                                                             s_q, heads, n_new, max_pages, num_pages, causal, scale, dst,
-                                                             lse, status_ws);
+  auto go = [&](auto fp8_tag, auto rpw_tag) {
+    var6_new_kernel<decltype(fp8_tag)::value, decltype(rpw_tag)::value><<<grid, kVarThreads, 0, stream>>>(
+        qq, kk, vv, pp, block_table, seqlens, oo, ool, lse_old, s_q, heads, n_new, max_pages, num_pages, causal,
+        scale, dst, lse, status_ws);
+  };
+  auto by_rows = [&](auto fp8_tag) {
+    const int rpw = (s_q + kVarWarps - 1) / kVarWarps;
+    if (rpw <= 1) go(fp8_tag, std::integral_constant<int, 1>{});
+    else if (rpw <= 2) go(fp8_tag, std::integral_constant<int, 2>{});
+    else if (rpw <= 4) go(fp8_tag, std::integral_constant<int, 4>{});
+    else go(fp8_tag, std::integral_constant<int, kMaxRowsPerWarp>{});
+  };
+  if (fp8) by_rows(std::true_type{});
+  else by_rows(std::false_type{});
   return cudaGetLastError();
 }
 
