@@ -234,21 +234,42 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
     transfers, pipelined over three streams (upload, compute, download).
     With three buffer sets a step's upload never waits for the download of
     the step before last, so uploads and downloads each run back to back on
-    their own copy engine."""
+    their own copy engine.  A step's inputs (query rows, block table,
+    lengths) travel as one packed copy and its outputs (O, lse) as one: the
+    library takes views into the packed device buffers, so each direction
+    pays one copy's fixed cost per step."""
     import mla_latent_space_b200 as mla
     nbuf = args.e2e_buffers
-    h_q = wl.q.pin_memory()
-    h_bt = torch.from_numpy(wl.block_table).pin_memory()
-    h_sl = torch.from_numpy(wl.seqlens).pin_memory()
+
+    def layout(parts):   # [(name, nbytes)] -> offsets 256-byte aligned, total
+        off, out = 0, {}
+        for name, nb in parts:
+            out[name] = (off, nb)
+            off = (off + nb + 255) // 256 * 256
+        return out, off
+
     oshape = (wl.batch, wl.s_q, wl.num_heads, 512)
     lshape = (wl.batch, wl.s_q, wl.num_heads)
-    h_out = [torch.empty(oshape, dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
-    h_lse = [torch.empty(lshape, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
-    d_q = [torch.empty_like(h_q, device=dev) for _ in range(nbuf)]
-    d_bt = [torch.empty_like(h_bt, device=dev) for _ in range(nbuf)]
-    d_sl = [torch.empty_like(h_sl, device=dev) for _ in range(nbuf)]
-    d_out = [torch.empty(oshape, dtype=torch.bfloat16, device=dev) for _ in range(nbuf)]
-    d_lse = [torch.empty(lshape, dtype=torch.float32, device=dev) for _ in range(nbuf)]
+    bt_np, sl_np = np.ascontiguousarray(wl.block_table), np.ascontiguousarray(wl.seqlens)
+    lin, nin = layout([("q", wl.q.numel() * 2), ("bt", bt_np.nbytes), ("sl", sl_np.nbytes)])
+    lout, nout = layout([("out", int(np.prod(oshape)) * 2), ("lse", int(np.prod(lshape)) * 4)])
+
+    def view(buf, lay, name, dtype, shp):
+        o, nb = lay[name]
+        return buf[o:o + nb].view(dtype).view(shp)
+
+    h_in = torch.empty(nin, dtype=torch.uint8).pin_memory()
+    view(h_in, lin, "q", torch.bfloat16, tuple(wl.q.shape)).copy_(wl.q)
+    view(h_in, lin, "bt", torch.int32, bt_np.shape).copy_(torch.from_numpy(bt_np))
+    view(h_in, lin, "sl", torch.int32, sl_np.shape).copy_(torch.from_numpy(sl_np))
+    h_out = [torch.empty(nout, dtype=torch.uint8).pin_memory() for _ in range(nbuf)]
+    d_in = [torch.empty(nin, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
+    d_outb = [torch.empty(nout, dtype=torch.uint8, device=dev) for _ in range(nbuf)]
+    d_q = [view(d, lin, "q", torch.bfloat16, tuple(wl.q.shape)) for d in d_in]
+    d_bt = [view(d, lin, "bt", torch.int32, bt_np.shape) for d in d_in]
+    d_sl = [view(d, lin, "sl", torch.int32, sl_np.shape) for d in d_in]
+    d_out = [view(d, lout, "out", torch.bfloat16, oshape) for d in d_outb]
+    d_lse = [view(d, lout, "lse", torch.float32, lshape) for d in d_outb]
     decs = [mla.Decoder(shape, device=dev) for _ in range(nbuf)]
     s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()
@@ -262,9 +283,7 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
         with torch.cuda.stream(s_up):
             if used[b]:
                 s_up.wait_event(down_done[b])       # its previous step is downloaded (so computed)
-            d_q[b].copy_(h_q, non_blocking=True)
-            d_bt[b].copy_(h_bt, non_blocking=True)
-            d_sl[b].copy_(h_sl, non_blocking=True)
+            d_in[b].copy_(h_in, non_blocking=True)
             up_done[b].record(s_up)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(up_done[b])
@@ -274,8 +293,7 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
             comp_done[b].record(s_comp)
         with torch.cuda.stream(s_down):
             s_down.wait_event(comp_done[b])
-            h_out[b].copy_(d_out[b], non_blocking=True)
-            h_lse[b].copy_(d_lse[b], non_blocking=True)
+            h_out[b].copy_(d_outb[b], non_blocking=True)
             down_done[b].record(s_down)
         used[b] = True
 
@@ -304,7 +322,10 @@ def run_e2e_pipelined(args, wl, dev, shape, pool, kv_scale, world):
     t1.record(s_up)
     torch.cuda.synchronize()
     barrier(world)
-    return max_over_ranks(t0.elapsed_time(t1) / K, world)
+    last = view(h_out[(K - 1) % nbuf], lout, "out", torch.bfloat16, oshape)
+    if not bool(torch.isfinite(last.float()).all()):
+        raise RuntimeError("non-finite output in the end-to-end loop")
+    return max_over_ranks(t0.elapsed_time(t1) / K, world), nin, nout
 
 
 def extra_steps(args):
@@ -758,7 +779,7 @@ def run_ours(args, wl, world, rank, local):
     # overlap step k+1's upload and step k-1's download (a step's kernels
     # wait for its upload; a buffer is reused only after the step that last
     # used it has been downloaded).  The cache (302 MB) is larger than L2.
-    e2e_ms = run_e2e_pipelined(args, wl, dev, dw.shape, dw.pool, dw.kv_scale, world)
+    e2e_ms, h2d, d2h = run_e2e_pipelined(args, wl, dev, dw.shape, dw.pool, dw.kv_scale, world)
     # the extras (the other workloads and the rows around the decode) are
     # timed in single-GPU runs; a multi-GPU run measures the headline step on
     # every replica
@@ -768,8 +789,6 @@ def run_ours(args, wl, world, rank, local):
         if extras and not args.no_projections else None
     sparse = run_sparse(args, dev, flush, pk) if extras and not args.no_sparse else None
     var6 = run_var6(args, dev, flush, pk) if extras and not args.no_var6 else None
-    h2d = wl.q.numel() * 2 + wl.block_table.size * 4 + wl.seqlens.size * 4
-    d2h = wl.batch * wl.s_q * wl.num_heads * (512 * 2 + 4)
     del dw
     torch.cuda.empty_cache()
     pcfg, pc_launches = per_config(args, dev, flush, pk, pk_kind, headline=(wl, step_ms, dec_ms, clk)) \
@@ -788,7 +807,8 @@ def run_ours(args, wl, world, rank, local):
             "clocks": clk,
             "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                    "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers"},
+                    "pipelining": f"upload / compute / download streams, {args.e2e_buffers} buffers, one packed "
+                                  "copy per direction"},
             "gpu_launches": 6 * K,
             "gpu_launches_note": "schedule + decode + combine, twice per timed iteration (the step timed whole, "
                                  "then with events around the decode launch)"}
