@@ -393,6 +393,11 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   return v;
 }
 
+// BF16 cache: V chunks per converter thread loaded together before their
+// stores (decode launch at b=64, h=128, t=4096: 116.7 us one at a time,
+// 111.4 us in groups of 4, 112.6 us with 8, 117.8 us with 16).
+constexpr int kConvGroup = 4;
+
 // Output CTA: the eight converter warps (-1 for other warps).  None shares a
 // scheduler sub-partition (warp % 4) with the PV issuer (warp 1): their
 // bursts of shared-memory loads would delay the issuer's barrier polls.
@@ -1245,21 +1250,30 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             }
           } else {
             if (!wwait(ctl, bar(bars->v_loaded[vs]), vph)) return false;
+            // Loads go out in groups of kConvGroup ahead of the group's
+            // stores (a thread's 16 chunks are its own, so the order is
+            // free): the shared-memory load latency is paid once per group
+            // instead of once per chunk.
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const uint32_t off = uint32_t(ct + kConvThreads * u) * 16u;
-              const int tok = int((off & (kBox - 1)) >> 7);
-              const uint4 v = ld_shared_v4(st + off);
-              if (tok < nvalid) {
-                const uint32_t a = bf16x2_to_f16x2(v.x), b = bf16x2_to_f16x2(v.y);
-                const uint32_t c = bf16x2_to_f16x2(v.z), d = bf16x2_to_f16x2(v.w);
-                track_absmax(vmax, a);
-                track_absmax(vmax, b);
-                track_absmax(vmax, c);
-                track_absmax(vmax, d);
-                st_shared_v4(st + off, a, b, c, d);
-              } else {
-                st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+            for (int u0 = 0; u0 < 16; u0 += kConvGroup) {
+              uint4 v[kConvGroup];
+#pragma unroll
+              for (int k = 0; k < kConvGroup; ++k) v[k] = ld_shared_v4(st + uint32_t(ct + kConvThreads * (u0 + k)) * 16u);
+#pragma unroll
+              for (int k = 0; k < kConvGroup; ++k) {
+                const uint32_t off = uint32_t(ct + kConvThreads * (u0 + k)) * 16u;
+                const int tok = int((off & (kBox - 1)) >> 7);
+                if (tok < nvalid) {
+                  const uint32_t a = bf16x2_to_f16x2(v[k].x), b = bf16x2_to_f16x2(v[k].y);
+                  const uint32_t c = bf16x2_to_f16x2(v[k].z), d = bf16x2_to_f16x2(v[k].w);
+                  track_absmax(vmax, a);
+                  track_absmax(vmax, b);
+                  track_absmax(vmax, c);
+                  track_absmax(vmax, d);
+                  st_shared_v4(st + off, a, b, c, d);
+                } else {
+                  st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+                }
               }
             }
           }
