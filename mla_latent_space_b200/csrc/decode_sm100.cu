@@ -51,6 +51,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "decode_launch.cuh"
 #include "kernel_util.cuh"
@@ -1253,29 +1254,40 @@ decode_sm100_kernel(const __grid_constant__ CUtensorMap pool_map, const __grid_c
             // Loads go out in groups of kConvGroup ahead of the group's
             // stores (a thread's 16 chunks are its own, so the order is
             // free): the shared-memory load latency is paid once per group
-            // instead of once per chunk.
+            // instead of once per chunk.  Chunk u of this thread holds token
+            // ct / 8 + 32 (u & 1).  A page whose 64 tokens all count (every
+            // page but a request's last, and valid) takes the loop without
+            // the per-token test; the CTA's converters all agree on it.  The
+            // converters are issue-bound: dropping the test took the b=64,
+            // h=128, t=4096 decode from 111.1 to 104.8 us.
+            auto convert = [&](auto masked) {
+              constexpr bool kMasked = decltype(masked)::value;
+              const bool va = (ct >> 3) < nvalid, vb = (ct >> 3) + 32 < nvalid;
 #pragma unroll
-            for (int u0 = 0; u0 < 16; u0 += kConvGroup) {
-              uint4 v[kConvGroup];
+              for (int u0 = 0; u0 < 16; u0 += kConvGroup) {
+                uint4 v[kConvGroup];
 #pragma unroll
-              for (int k = 0; k < kConvGroup; ++k) v[k] = ld_shared_v4(st + uint32_t(ct + kConvThreads * (u0 + k)) * 16u);
+                for (int k = 0; k < kConvGroup; ++k)
+                  v[k] = ld_shared_v4(st + uint32_t(ct + kConvThreads * (u0 + k)) * 16u);
 #pragma unroll
-              for (int k = 0; k < kConvGroup; ++k) {
-                const uint32_t off = uint32_t(ct + kConvThreads * (u0 + k)) * 16u;
-                const int tok = int((off & (kBox - 1)) >> 7);
-                if (tok < nvalid) {
-                  const uint32_t a = bf16x2_to_f16x2(v[k].x), b = bf16x2_to_f16x2(v[k].y);
-                  const uint32_t c = bf16x2_to_f16x2(v[k].z), d = bf16x2_to_f16x2(v[k].w);
-                  track_absmax(vmax, a);
-                  track_absmax(vmax, b);
-                  track_absmax(vmax, c);
-                  track_absmax(vmax, d);
-                  st_shared_v4(st + off, a, b, c, d);
-                } else {
-                  st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+                for (int k = 0; k < kConvGroup; ++k) {
+                  const uint32_t off = uint32_t(ct + kConvThreads * (u0 + k)) * 16u;
+                  if (!kMasked || (((u0 + k) & 1) ? vb : va)) {
+                    const uint32_t a = bf16x2_to_f16x2(v[k].x), b = bf16x2_to_f16x2(v[k].y);
+                    const uint32_t c = bf16x2_to_f16x2(v[k].z), d = bf16x2_to_f16x2(v[k].w);
+                    track_absmax(vmax, a);
+                    track_absmax(vmax, b);
+                    track_absmax(vmax, c);
+                    track_absmax(vmax, d);
+                    st_shared_v4(st + off, a, b, c, d);
+                  } else {
+                    st_shared_v4(st + off, 0u, 0u, 0u, 0u);
+                  }
                 }
               }
-            }
+            };
+            if (nvalid >= MLA_PAGE_SIZE) convert(std::false_type{});
+            else convert(std::true_type{});
           }
           fence_proxy_async_cta();
           mbar_arrive(bar(bars->v_full[vs]));
